@@ -1,0 +1,433 @@
+#!/usr/bin/env python3
+"""Benchmark of the ternary GEMM (TQ2/TQ1 packed weights x fp16 activations).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--sweep]
+
+One step = one pass of the ternary linear layers of the workload over one
+batch of synthetic activations (weights are prepared once, as the pages
+describe: "At inference, only W_hat and gamma are stored").  The default
+workload is the single-layer decode GEMV set of a LLaMA-7B-like model
+(W in {4096x4096, 11008x4096, 4096x11008}, M = 1, TQ2).  Weights are
+absmean-ternarized from N(0, 0.02) latent weights by this library, then
+cloned into enough rotating copies that every timed step reads weights that
+are not in L2 (the copies total > 3x the L2 size).  The timed region replays
+one CUDA graph per step; events inside the graphs time every GEMM launch.
+
+Prints ONE JSON line (rank 0).  With --sweep, writes a table of lines for
+the batch sweep, the 70B-like block and the sparsity stress workloads.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# ------------------------------------------------------------------ workloads
+WORKLOADS = {
+    # single-layer decode GEMV, LLaMA-7B-like shapes, M = 1 (N, K per layer)
+    "llama7b_decode_m1": dict(layers=[(4096, 4096), (11008, 4096), (4096, 11008)], M=1, fmt="tq2",
+                              seeds=[2, 3, 4]),
+    "down_8192x28672_m1": dict(layers=[(8192, 28672)], M=1, fmt="tq2", seeds=[16]),
+    "square_8192_m256": dict(layers=[(8192, 8192)], M=256, fmt="tq2", seeds=[5]),
+    # 70B-like block linears at batch 16: q, k, v, o, gate, up, down
+    "block70b_m16": dict(layers=[(8192, 8192), (1024, 8192), (1024, 8192), (8192, 8192),
+                                 (28672, 8192), (28672, 8192), (8192, 28672)], M=16, fmt="tq2",
+                         seeds=[10, 11, 12, 13, 14, 15, 16]),
+}
+KERNELS_PER_CALL = {1: 1, 2: 2, 3: 1}   # path -> launches of this library's kernels per GEMM
+
+
+def workload_from_args(name, M=None, fmt=None):
+    w = dict(WORKLOADS[name])
+    if M is not None:
+        w["M"] = M
+    if fmt is not None:
+        w["fmt"] = fmt
+    w["name"] = name
+    return w
+
+
+def algo_bytes(fmt, M, N, K):
+    from bit_mixed_precision_tri_b200.api import packed_row_bytes
+    return N * packed_row_bytes(fmt, K) + N * (K // 256) * 2 + M * K * 2 + M * N * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {k: float(j[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    cs = os.path.join(ROOT, "bit_mixed_precision_tri_b200", "csrc")
+    for fn in sorted(os.listdir(cs)):
+        with open(os.path.join(cs, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the
+    current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src = kernel_source_hash()
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel \
+                    and parts[1] == src and parts[3] == workload:
+                return float(parts[2])
+    return None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 8:
+                continue
+            try:
+                sm.append(float(p[0]))
+                mx.append(float(p[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def prepare_layers(w, device, copies):
+    import bit_mixed_precision_tri_b200 as tri
+    from bit_mixed_precision_tri_b200 import inputs
+    layers = []
+    for (N, K), seed in zip(w["layers"], w["seeds"]):
+        W = inputs.latent_weights(N, K, seed).to(device)
+        trits, g = tri.ternarize(W, 1e-6)
+        qs, d = tri.pack(trits, g, w["fmt"])
+        del W, trits
+        reps = [(qs, d)] + [(qs.clone(), d.clone()) for _ in range(copies - 1)]
+        X = inputs.activations(w["M"], K, 6 + w["M"] + seed).to(device)
+        Y = torch.empty(w["M"], N, dtype=torch.float16, device=device)
+        layers.append(dict(N=N, K=K, reps=reps, X=X, Y=Y, gamma=float(g.item())))
+    torch.cuda.synchronize(device)
+    return layers
+
+
+def run_ours(args, rank, world, device):
+    import bit_mixed_precision_tri_b200 as tri
+    w = workload_from_args(args.workload, args.M, args.fmt)
+    M, fmt = w["M"], w["fmt"]
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    step_bytes = sum(algo_bytes(fmt, M, N, K) for N, K in w["layers"])
+    weight_bytes = sum(N * tri.packed_row_bytes(fmt, K) + N * (K // 256) * 2 for N, K in w["layers"])
+    copies = max(args.steps, int(np.ceil(3 * l2 / max(weight_bytes, 1))) + 1)
+    layers = prepare_layers(w, device, copies)
+    paths = [tri.auto_path(fmt, M, L["N"], L["K"]) for L in layers]
+    ws = tri.Workspace(device)
+    ws.get(max(tri.gemm_workspace_bytes(fmt, M, L["N"], L["K"]) for L in layers))
+    stream = torch.cuda.Stream(device)
+
+    def step(c, evs=None):
+        for i, L in enumerate(layers):
+            qs, d = L["reps"][c]
+            if evs is not None:
+                evs[i][0].record(stream)
+            tri.gemm(L["X"], qs, d, L["N"], L["K"], fmt, out=L["Y"], workspace=ws, stream=stream)
+            if evs is not None:
+                evs[i][1].record(stream)
+
+    # eager warm-up (also allocates), then one graph per copy
+    with torch.cuda.stream(stream):
+        for c in range(min(copies, 2)):
+            step(c)
+    torch.cuda.synchronize(device)
+    graphs, events = [], []
+    for c in range(copies):
+        evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                torch.cuda.Event(enable_timing=True, external=True)) for _ in layers]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(c, evs)
+        graphs.append(g)
+        events.append(evs)
+    torch.cuda.synchronize(device)
+    for i in range(args.warmup):
+        graphs[(copies - 1 - i) % copies].replay()
+    torch.cuda.synchronize(device)
+
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for s in range(args.steps):
+            graphs[s % copies].replay()
+        t1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    clk = clocks.stop() if rank == 0 else None
+    elapsed_ms = t0.elapsed_time(t1)
+    per_launch = []   # (bytes, ms) of every GEMM launch in the timed region
+    for s in range(min(args.steps, copies)):
+        for i, L in enumerate(layers):
+            a, b = events[s][i]
+            per_launch.append((algo_bytes(fmt, M, L["N"], L["K"]), a.elapsed_time(b)))
+    kernel_ms = sum(ms for _, ms in per_launch)
+    kernel_bytes = sum(b for b, _ in per_launch)
+    max_ms = allreduce_max(elapsed_ms, world, device)
+
+    # end-to-end through the public API: pinned host X -> device, GEMM, Y -> host
+    xh = [L["X"].cpu().pin_memory() for L in layers]
+    yh = [torch.empty(M, L["N"], dtype=torch.float16).pin_memory() for L in layers]
+    xd = [torch.empty_like(L["X"]) for L in layers]
+    h2d = sum(x.numel() * 2 for x in xh)
+    d2h = sum(y.numel() * 2 for y in yh)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for rep in range(2):   # first pass warms, second is timed
+            if rep == 1:
+                barrier(world)
+                torch.cuda.synchronize(device)
+                e0.record(stream)
+            for s in range(args.steps):
+                c = s % copies
+                for i, L in enumerate(layers):
+                    xd[i].copy_(xh[i], non_blocking=True)
+                    qs, d = L["reps"][c]
+                    tri.gemm(xd[i], qs, d, L["N"], L["K"], fmt, out=L["Y"], workspace=ws,
+                             stream=stream)
+                    yh[i].copy_(L["Y"], non_blocking=True)
+            if rep == 1:
+                e1.record(stream)
+            torch.cuda.synchronize(device)
+    e2e_ms = allreduce_max(e0.elapsed_time(e1), world, device)
+    del graphs
+    launches = args.steps * sum(KERNELS_PER_CALL.get(p, 1) for p in paths)
+    unit = "GB/s" if M <= 32 else "TFLOP/s"
+    flops = sum(2.0 * M * N * K for N, K in w["layers"])
+
+    def metric_value(ms, steps):
+        if unit == "GB/s":
+            return world * steps * step_bytes / (ms * 1e-3) / 1e9
+        return world * steps * flops / (ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    if unit == "GB/s":
+        achieved = kernel_bytes / (kernel_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src,
+                "traffic": recorded_traffic("gemm", w["name"])}
+    else:
+        kflops = sum(2.0 * M * L["N"] * L["K"] for L in layers) * min(args.steps, copies)
+        achieved = kflops / (kernel_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "peak_source": peak_src,
+                "traffic": recorded_traffic("gemm", w["name"])}
+    roof["kernel_launches_timed"] = len(per_launch)
+    roof["kernel_ms_per_launch"] = kernel_ms / max(len(per_launch), 1)
+    res = {
+        "metric": "TQ2/TQ1 ternary GEMM: HBM GB/s (M<=16) and TFLOP/s (M>=64) vs roofline",
+        "value": metric_value(max_ms, args.steps),
+        "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16xternary->f32acc",
+        "data": "synthetic",
+        "config": {"workload": w["name"], "layers_NxK": [f"{N}x{K}" for N, K in w["layers"]],
+                   "M": M, "format": fmt, "global_batch": M * world,
+                   "paths": paths, "weight_copies": copies,
+                   "l2_policy": f"rotating {copies} weight copies ({copies * weight_bytes / 1e6:.0f} MB > 3x L2)",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "roofline": roof,
+        "e2e": {"value": metric_value(e2e_ms, args.steps), "unit": unit,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    return res
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample(w, budget_s=12.0):
+    """Time the CPU oracle (as it stands) on a bounded sample of the workload:
+    whole layers (unpack + fp64 GEMM) until ~budget_s of CPU work; returns
+    (value in the workload's unit, description, threads)."""
+    from bit_mixed_precision_tri_b200 import inputs
+    from oracle import tri_oracle as O
+    M, fmt = w["M"], w["fmt"]
+    unit = "GB/s" if M <= 32 else "TFLOP/s"
+    prepared = []
+    for (N, K), seed in zip(w["layers"], w["seeds"]):
+        rows = min(N, 2048)
+        W = inputs.latent_weights(rows, K, seed).numpy()
+        t, g = O.absmean_ternarize(W, 1e-6)
+        qs, d = O.pack(fmt, t, np.array([g], np.float32))
+        X = inputs.activations(M, K, 6 + M + seed).numpy()
+        prepared.append((rows, K, qs, d, X))
+    done_bytes = done_flops = 0.0
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        for rows, K, qs, d, X in prepared:
+            O.gemm_packed_f64(fmt, X, qs, d, rows, K)
+            done_bytes += algo_bytes(fmt, M, rows, K)
+            done_flops += 2.0 * M * rows * K
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    val = done_bytes / dt / 1e9 if unit == "GB/s" else done_flops / dt / 1e12
+    desc = (f"{n} passes over the first min(N, 2048) rows of each layer "
+            f"({'+'.join(str(min(N, 2048)) + 'x' + str(K) for N, K in w['layers'])}), "
+            f"unpack + float64 GEMM, {dt:.1f} s")
+    try:
+        threads = len(os.sched_getaffinity(0))
+    except Exception:
+        threads = os.cpu_count()
+    return val, unit, desc, threads
+
+
+def run_reference(args, rank, world):
+    w = workload_from_args(args.workload, args.M, args.fmt)
+    if rank != 0:
+        return None
+    budget = max(3.0, 60.0 / max(args.steps + args.warmup, 1))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, unit, desc, threads = oracle_sample(w, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference",
+        "metric": "TQ2/TQ1 ternary GEMM: HBM GB/s (M<=16) and TFLOP/s (M>=64) vs roofline",
+        "value": value, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": budget * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w["name"], "layers_NxK": [f"{N}x{K}" for N, K in w["layers"]],
+                   "M": w["M"], "format": w["fmt"]},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------ dist utils
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def allreduce_max(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama7b_decode_m1", choices=sorted(WORKLOADS))
+    ap.add_argument("--M", type=int, default=None)
+    ap.add_argument("--fmt", default=None, choices=[None, "tq2", "tq1"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if world > 1 and rank != 0:
+            return
+        res = run_reference(args, 0, world)
+        print(json.dumps(res), flush=True)
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        res = run_ours(args, rank, world, device)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            w = workload_from_args(args.workload, args.M, args.fmt)
+            v, unit, desc, threads = oracle_sample(w, budget_s=10.0)
+            res["cpu_baseline"] = {"value": v, "unit": unit, "cores": threads, "kind": "oracle",
+                                   "sample": desc}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+"""Torch-facing wrappers over the C ABI (include/tri.h).
+
+PyTorch provides device memory and the current CUDA stream; every step of the
+path runs in the library's CUDA kernels.  Functions raise ``TriError`` on a
+non-OK status and never fall back to another implementation.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import PATH_AUTO, PATH_MMA, PATH_SIMT, PATH_TCGEN05, TRI_TQ1, TRI_TQ2, TriError  # noqa: F401
+
+FORMATS = {"tq2": TRI_TQ2, "tq1": TRI_TQ1}
+
+
+def _fmt(fmt) -> int:
+    if isinstance(fmt, str):
+        return FORMATS[fmt]
+    return int(fmt)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def packed_row_bytes(fmt, K: int) -> int:
+    return K // 4 if _fmt(fmt) == TRI_TQ2 else (K // 256) * 52
+
+
+# ------------------------------------------------------------------ a1, a2
+def absmean(W: torch.Tensor, eps: float = 1e-6) -> torch.Tensor:
+    """gamma = eps + mean|W| (exact sum), as a device float32 tensor of shape (1,)."""
+    _require_cuda(W)
+    N, K = W.shape
+    L = _lib.lib()
+    ws = torch.empty(L.tri_absmean_workspace_bytes(N, K), dtype=torch.uint8, device=W.device)
+    g = torch.empty(1, dtype=torch.float32, device=W.device)
+    _lib.check(L.tri_absmean(_ptr(W), N, K, eps, _ptr(g), _ptr(ws), ws.numel(), _stream(W.device)),
+               "tri_absmean")
+    return g
+
+
+def ternarize(W: torch.Tensor, eps: float = 1e-6, check_finite: bool = True):
+    """(trits int8[N][K], gamma float32[1]) by absmean ternarization.
+
+    With ``check_finite`` the host waits for gamma and raises TriError
+    (TRI_ERR_NONFINITE) when W held Inf or NaN.
+    """
+    _require_cuda(W)
+    if W.dtype != torch.float32:
+        raise ValueError("W must be float32")
+    N, K = W.shape
+    L = _lib.lib()
+    ws = torch.empty(L.tri_absmean_workspace_bytes(N, K), dtype=torch.uint8, device=W.device)
+    g = torch.empty(1, dtype=torch.float32, device=W.device)
+    trits = torch.empty(N, K, dtype=torch.int8, device=W.device)
+    _lib.check(L.tri_ternarize(_ptr(W), N, K, eps, _ptr(trits), _ptr(g), _ptr(ws), ws.numel(),
+                               _stream(W.device)), "tri_ternarize")
+    if check_finite and not torch.isfinite(g).item():
+        raise TriError(4, "tri_ternarize: weights hold Inf or NaN")
+    return trits, g
+
+
+# ------------------------------------------------------------------ a3, a4
+def pack(trits: torch.Tensor, scales: torch.Tensor, fmt="tq2", return_invalid: bool = False):
+    """(qs uint8, d fp16[N][K/256]) in TQ2 or TQ1.  ``scales`` is float32 of
+    one element (one scale for the matrix) or N*K/256 elements (per block)."""
+    _require_cuda(trits, scales)
+    N, K = trits.shape
+    f = _fmt(fmt)
+    qs = torch.empty(N, packed_row_bytes(f, K), dtype=torch.uint8, device=trits.device)
+    d = torch.empty(N, K // 256, dtype=torch.float16, device=trits.device)
+    inv = torch.zeros(1, dtype=torch.int32, device=trits.device)
+    fn = _lib.lib().tri_pack_tq2 if f == TRI_TQ2 else _lib.lib().tri_pack_tq1
+    _lib.check(fn(_ptr(trits), N, K, _ptr(scales), scales.numel(), _ptr(qs), _ptr(d), _ptr(inv),
+                  _stream(trits.device)), "tri_pack")
+    return (qs, d, inv) if return_invalid else (qs, d)
+
+
+def unpack(qs: torch.Tensor, N: int, K: int, fmt="tq2", return_invalid: bool = False):
+    """int8 trits[N][K] decoded from a packed plane."""
+    _require_cuda(qs)
+    trits = torch.empty(N, K, dtype=torch.int8, device=qs.device)
+    inv = torch.zeros(1, dtype=torch.int32, device=qs.device)
+    _lib.check(_lib.lib().tri_unpack(_fmt(fmt), _ptr(qs), N, K, _ptr(trits), _ptr(inv),
+                                     _stream(qs.device)), "tri_unpack")
+    return (trits, inv) if return_invalid else trits
+
+
+# ------------------------------------------------------------------ a6
+def gemm_workspace_bytes(fmt, M: int, N: int, K: int) -> int:
+    return int(_lib.lib().tri_gemm_workspace_bytes(_fmt(fmt), M, N, K))
+
+
+def auto_path(fmt, M: int, N: int, K: int) -> int:
+    return int(_lib.lib().tri_gemm_auto_path(_fmt(fmt), M, N, K))
+
+
+class Workspace:
+    """Zero-filled device scratch for tri_gemm, grown on demand (kept zeroed
+    by the kernels between calls)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _workspace_for(device) -> Workspace:
+    key = torch.device(device)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(key)
+    return _default_ws[key]
+
+
+def gemm(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, N: int, K: int, fmt="tq2",
+         path: int = PATH_AUTO, out: torch.Tensor = None, workspace: Workspace = None,
+         stream=None) -> torch.Tensor:
+    """Y = X (d * W_hat)^T in fp16 with fp32 accumulation."""
+    _require_cuda(X, qs, d)
+    if X.dtype != torch.float16:
+        raise ValueError("X must be float16")
+    M = X.shape[0]
+    f = _fmt(fmt)
+    Y = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=X.device)
+    ws = (workspace or _workspace_for(X.device)).get(gemm_workspace_bytes(f, M, N, K))
+    s = stream.cuda_stream if stream is not None else _stream(X.device)
+    _lib.check(_lib.lib().tri_gemm(f, int(path), _ptr(X), _ptr(qs), _ptr(d), _ptr(Y), M, N, K,
+                                   _ptr(ws), ws.numel(), s), "tri_gemm")
+    return Y
+
+
+class TernaryLinear:
+    """A ternary linear layer: absmean-ternarized, packed weights and a GEMM.
+
+    ``TernaryLinear.from_latent(W)`` ternarizes latent float32 weights on the
+    GPU, packs them (TQ2 or TQ1) with d = fp16(gamma) in every block, and
+    ``layer(X)`` computes X (gamma W_hat)^T.
+    """
+
+    def __init__(self, qs, d, N, K, fmt="tq2", gamma=None):
+        self.qs, self.d, self.N, self.K, self.fmt, self.gamma = qs, d, N, K, fmt, gamma
+        self.ws = Workspace(qs.device)
+
+    @classmethod
+    def from_latent(cls, W: torch.Tensor, fmt="tq2", eps: float = 1e-6):
+        trits, g = ternarize(W, eps)
+        qs, d = pack(trits, g, fmt)
+        return cls(qs, d, W.shape[0], W.shape[1], fmt, g)
+
+    def __call__(self, X: torch.Tensor, path: int = PATH_AUTO, out=None) -> torch.Tensor:
+        return gemm(X, self.qs, self.d, self.N, self.K, self.fmt, path=path, out=out,
+                    workspace=self.ws)

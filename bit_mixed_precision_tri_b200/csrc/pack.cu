@@ -1,0 +1,233 @@
+// TQ2 / TQ1 packing and unpacking on sm_100a.
+//
+// "Scaling Laws and Efficient Inference for Ternary Language Models",
+// section "Packing ternary weights":
+//   * every weight d in {-1,0,1} is shifted to d' = d + 1 in {0,1,2};
+//   * "2 bits per weight": four digits per byte, decoded by a shift and a mask
+//     d' = (b >> 2j) & 3; with the "TriRun" storage line (sixteen 2-bit weights
+//     per 32-bit word) this library puts weight j of a 16-weight word at bits 2j;
+//   * "1.6 bits per weight": five digits read as a base-3 number N5 (first
+//     weight most significant) become the byte floor((256*N5 + 242)/243);
+//     decoding multiplies by 3 and splits off the high byte as the next digit.
+// Section "Fast inference on CPUs": 256-weight blocks with one 16-bit scale.
+//
+// TQ1 block layout (52 bytes per 256 weights): bytes 0..50 hold weights
+// 5g..5g+4 of the block, byte 51 holds weight 255 followed by four zero
+// weights (digit 1 each).
+//
+// All four kernels are byte streams bound by HBM bandwidth; one thread packs
+// or unpacks one 32-bit TQ2 word (16 weights) or one TQ1 byte (5 weights).
+#include "tri_internal.cuh"
+
+namespace tri {
+namespace {
+
+constexpr int kThreads = 256;
+
+int grid_for(int64_t items) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t g = ceil_div(items, kThreads);
+  const int64_t cap = (int64_t)sms * 16;
+  if (g > cap) g = cap;
+  return (int)(g < 1 ? 1 : g);
+}
+
+__device__ __forceinline__ void block_count_add(int cnt, int32_t* counter) {
+  // warp reduce, then one atomic per warp
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, o);
+  if ((threadIdx.x & 31) == 0 && cnt != 0 && counter != nullptr) atomicAdd(counter, cnt);
+}
+
+// digit d' of a trit byte; values outside {-1,0,1} count as invalid, packed as 0
+__device__ __forceinline__ unsigned digit_of(int8_t t, int& bad) {
+  const int v = (int)t;
+  if (v < -1 || v > 1) { ++bad; return 1u; }
+  return (unsigned)(v + 1);
+}
+
+__global__ void __launch_bounds__(kThreads)
+pack_tq2_kernel(const int8_t* __restrict__ trits, int64_t nwords, uint32_t* __restrict__ qs,
+                int32_t* invalid) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nwords; base += stride, i += stride) {
+    int bad = 0;
+    if (i < nwords) {
+      const uint4 v = reinterpret_cast<const uint4*>(trits)[i];
+      const unsigned w4[4] = {v.x, v.y, v.z, v.w};
+      unsigned word = 0u;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int8_t t = (int8_t)((w4[q] >> (8 * b)) & 0xFFu);
+          word |= digit_of(t, bad) << (2 * (4 * q + b));
+        }
+      qs[i] = word;
+    }
+    block_count_add(bad, invalid);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+pack_tq1_kernel(const int8_t* __restrict__ trits, int64_t N, int64_t K, uint8_t* __restrict__ qs,
+                int32_t* invalid) {
+  const int64_t nb = K / kBlock;
+  const int64_t nbytes = N * nb * kTq1BlockBytes;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nbytes; base += stride, i += stride) {
+    int bad = 0;
+    if (i < nbytes) {
+      const int64_t rowblk = i / kTq1BlockBytes;          // n * nb + b
+      const int j = (int)(i - rowblk * kTq1BlockBytes);
+      const int64_t n = rowblk / nb, b = rowblk - n * nb;
+      const int8_t* t = trits + n * K + b * kBlock + 5 * j;
+      unsigned n5 = 0u;
+      if (j < kTq1Groups) {
+#pragma unroll
+        for (int q = 0; q < 5; ++q) n5 = 3u * n5 + digit_of(t[q], bad);
+      } else {
+        n5 = digit_of(t[0], bad);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) n5 = 3u * n5 + 1u;     // four zero weights
+      }
+      qs[i] = (uint8_t)((n5 * 256u + 242u) / 243u);
+    }
+    block_count_add(bad, invalid);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+scales_kernel(const float* __restrict__ scales, int64_t n_scales, int64_t count,
+              __half* __restrict__ d) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < count; i += stride)
+    d[i] = __float2half_rn(scales[n_scales == 1 ? 0 : i]);
+}
+
+__global__ void __launch_bounds__(kThreads)
+unpack_tq2_kernel(const uint32_t* __restrict__ qs, int64_t nwords, int8_t* __restrict__ trits,
+                  int32_t* invalid) {
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nwords; base += stride, i += stride) {
+    int bad = 0;
+    if (i < nwords) {
+      const unsigned w = qs[i];
+      unsigned out[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        unsigned o = 0u;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const unsigned f = (w >> (2 * (4 * q + b))) & 3u;
+          bad += (f == 3u);
+          o |= ((f - 1u) & 0xFFu) << (8 * b);
+        }
+        out[q] = o;
+      }
+      reinterpret_cast<uint4*>(trits)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    block_count_add(bad, invalid);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+unpack_tq1_kernel(const uint8_t* __restrict__ qs, int64_t N, int64_t K, int8_t* __restrict__ trits,
+                  int32_t* invalid) {
+  const int64_t nb = K / kBlock;
+  const int64_t nbytes = N * nb * kTq1BlockBytes;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nbytes; base += stride, i += stride) {
+    int bad = 0;
+    if (i < nbytes) {
+      const int64_t rowblk = i / kTq1BlockBytes;
+      const int j = (int)(i - rowblk * kTq1BlockBytes);
+      const int64_t n = rowblk / nb, b = rowblk - n * nb;
+      const unsigned byte = qs[i];
+      // multiply-shift decoder: x*3, high byte is the digit, low byte goes on
+      unsigned v = byte, dig[5], n5 = 0u;
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        v *= 3u;
+        dig[q] = v >> 8;
+        v &= 0xFFu;
+        n5 = 3u * n5 + dig[q];
+      }
+      bad += ((n5 * 256u + 242u) / 243u) != byte;     // not in the encoder's image
+      int8_t* t = trits + n * K + b * kBlock + 5 * j;
+      if (j < kTq1Groups) {
+#pragma unroll
+        for (int q = 0; q < 5; ++q) t[q] = (int8_t)((int)dig[q] - 1);
+      } else {
+        t[0] = (int8_t)((int)dig[0] - 1);
+        bad += (dig[1] != 1u || dig[2] != 1u || dig[3] != 1u || dig[4] != 1u) &&
+               ((n5 * 256u + 242u) / 243u) == byte;
+      }
+    }
+    block_count_add(bad, invalid);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack_tq2(const int8_t* trits, int64_t N, int64_t K, const float* scales,
+                            int64_t n_scales, uint8_t* qs, uint16_t* d, int32_t* invalid,
+                            cudaStream_t s) {
+  if (invalid) {
+    cudaError_t e = cudaMemsetAsync(invalid, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t nwords = N * K / 16;
+  pack_tq2_kernel<<<grid_for(nwords), kThreads, 0, s>>>(trits, nwords,
+                                                         reinterpret_cast<uint32_t*>(qs), invalid);
+  const int64_t nd = N * (K / kBlock);
+  scales_kernel<<<grid_for(nd), kThreads, 0, s>>>(scales, n_scales, nd,
+                                                   reinterpret_cast<__half*>(d));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_tq1(const int8_t* trits, int64_t N, int64_t K, const float* scales,
+                            int64_t n_scales, uint8_t* qs, uint16_t* d, int32_t* invalid,
+                            cudaStream_t s) {
+  if (invalid) {
+    cudaError_t e = cudaMemsetAsync(invalid, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t nbytes = N * (K / kBlock) * kTq1BlockBytes;
+  pack_tq1_kernel<<<grid_for(nbytes), kThreads, 0, s>>>(trits, N, K, qs, invalid);
+  const int64_t nd = N * (K / kBlock);
+  scales_kernel<<<grid_for(nd), kThreads, 0, s>>>(scales, n_scales, nd,
+                                                   reinterpret_cast<__half*>(d));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_tq2(const uint8_t* qs, int64_t N, int64_t K, int8_t* trits,
+                              int32_t* invalid, cudaStream_t s) {
+  if (invalid) {
+    cudaError_t e = cudaMemsetAsync(invalid, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t nwords = N * K / 16;
+  unpack_tq2_kernel<<<grid_for(nwords), kThreads, 0, s>>>(
+      reinterpret_cast<const uint32_t*>(qs), nwords, trits, invalid);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_tq1(const uint8_t* qs, int64_t N, int64_t K, int8_t* trits,
+                              int32_t* invalid, cudaStream_t s) {
+  if (invalid) {
+    cudaError_t e = cudaMemsetAsync(invalid, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t nbytes = N * (K / kBlock) * kTq1BlockBytes;
+  unpack_tq1_kernel<<<grid_for(nbytes), kThreads, 0, s>>>(qs, N, K, trits, invalid);
+  return cudaGetLastError();
+}
+
+}  // namespace tri

@@ -1,0 +1,227 @@
+// The C ABI (include/tri.h): host-side validation and dispatch.
+//
+// Every entry point checks its arguments before enqueuing anything, launches
+// on the caller's stream, never allocates and never synchronizes.
+#include <mutex>
+
+#include "tri_internal.cuh"
+
+namespace {
+
+using tri::ceil_div;
+
+constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct DevInfo {
+  int sms = 0;
+  int major = 0;
+  int minor = 0;
+};
+
+constexpr int kMaxDevices = 64;
+DevInfo g_dev[kMaxDevices];
+std::once_flag g_once[kMaxDevices];
+
+tri_status device_info(DevInfo* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return TRI_ERR_CUDA;
+  }
+  std::call_once(g_once[dev], [dev]() {
+    cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&g_dev[dev].major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&g_dev[dev].minor, cudaDevAttrComputeCapabilityMinor, dev);
+  });
+  *out = g_dev[dev];
+  if (out->major != 10 || out->minor != 0) return TRI_ERR_NO_DEVICE;
+  return TRI_OK;
+}
+
+tri_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return TRI_OK;
+  cudaGetLastError();
+  return TRI_ERR_CUDA;
+}
+
+tri_status check_nk(int64_t N, int64_t K) {
+  if (N < 1 || K < tri::kBlock || K % tri::kBlock != 0) return TRI_ERR_SHAPE;
+  if (N > kMaxDim || K > kMaxDim) return TRI_ERR_SHAPE;
+  if (N * K >= (int64_t(1) << 40)) return TRI_ERR_SHAPE;
+  return TRI_OK;
+}
+
+int auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
+  if (M <= 16 && tri::gemv_mma_supported(fmt, M, N, K)) return TRI_PATH_MMA;
+  if (M >= 64 && tri::gemm_tc_supported(fmt, M, N, K)) return TRI_PATH_TCGEN05;
+  if (tri::gemm_tc_supported(fmt, M, N, K) && M > 16) return TRI_PATH_TCGEN05;
+  if (tri::gemv_mma_supported(fmt, M, N, K)) return TRI_PATH_MMA;
+  return TRI_PATH_SIMT;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tri_status_string(int status) {
+  switch (status) {
+    case TRI_OK: return "ok";
+    case TRI_ERR_INVALID_ARG: return "invalid argument";
+    case TRI_ERR_SHAPE: return "invalid shape (need N,M >= 1, K >= 256, K % 256 == 0)";
+    case TRI_ERR_ALIGNMENT: return "misaligned pointer";
+    case TRI_ERR_NONFINITE: return "non-finite weights";
+    case TRI_ERR_INVALID_CODE: return "invalid packed code";
+    case TRI_ERR_CUDA: return "CUDA runtime error";
+    case TRI_ERR_NOT_IMPLEMENTED: return "kernel path not available for this shape";
+    case TRI_ERR_WORKSPACE: return "workspace missing or too small";
+    case TRI_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    default: return "unknown status";
+  }
+}
+
+int tri_version(void) { return 100; }
+
+size_t tri_absmean_workspace_bytes(int64_t, int64_t) { return tri::absmean_ws_bytes(); }
+
+tri_status tri_absmean(const float* W, int64_t N, int64_t K, float eps, float* gamma,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!W || !gamma) return TRI_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || eps > 3.0e38f) return TRI_ERR_INVALID_ARG;
+  tri_status st = check_nk(N, K);
+  if (st != TRI_OK) return st;
+  if (!workspace || workspace_bytes < tri::absmean_ws_bytes()) return TRI_ERR_WORKSPACE;
+  if (!aligned(W, 16) || !aligned(workspace, 16) || !aligned(gamma, 4)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  if ((st = device_info(&di)) != TRI_OK) return st;
+  return from_cuda(tri::launch_absmean(W, N * K, eps, gamma, workspace,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+tri_status tri_ternarize(const float* W, int64_t N, int64_t K, float eps, int8_t* trits,
+                         float* gamma, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!trits) return TRI_ERR_INVALID_ARG;
+  if (!aligned(trits, 16)) return TRI_ERR_ALIGNMENT;
+  tri_status st = tri_absmean(W, N, K, eps, gamma, workspace, workspace_bytes, stream);
+  if (st != TRI_OK) return st;
+  return from_cuda(tri::launch_ternarize(W, N * K, gamma, trits, static_cast<cudaStream_t>(stream)));
+}
+
+static tri_status pack_common(int fmt, const int8_t* trits, int64_t N, int64_t K,
+                              const float* scales, int64_t n_scales, uint8_t* qs, uint16_t* d,
+                              int32_t* invalid_count, void* stream) {
+  if (!trits || !scales || !qs || !d) return TRI_ERR_INVALID_ARG;
+  tri_status st = check_nk(N, K);
+  if (st != TRI_OK) return st;
+  if (n_scales != 1 && n_scales != N * (K / tri::kBlock)) return TRI_ERR_INVALID_ARG;
+  if (!aligned(trits, 16) || !aligned(scales, 4) || !aligned(d, 4)) return TRI_ERR_ALIGNMENT;
+  if (!aligned(qs, fmt == TRI_TQ2 ? 16 : 4)) return TRI_ERR_ALIGNMENT;
+  if (invalid_count && !aligned(invalid_count, 4)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  if ((st = device_info(&di)) != TRI_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fmt == TRI_TQ2)
+    return from_cuda(tri::launch_pack_tq2(trits, N, K, scales, n_scales, qs, d, invalid_count, s));
+  return from_cuda(tri::launch_pack_tq1(trits, N, K, scales, n_scales, qs, d, invalid_count, s));
+}
+
+tri_status tri_pack_tq2(const int8_t* trits, int64_t N, int64_t K, const float* scales,
+                        int64_t n_scales, uint8_t* qs, uint16_t* d, int32_t* invalid_count,
+                        void* stream) {
+  return pack_common(TRI_TQ2, trits, N, K, scales, n_scales, qs, d, invalid_count, stream);
+}
+
+tri_status tri_pack_tq1(const int8_t* trits, int64_t N, int64_t K, const float* scales,
+                        int64_t n_scales, uint8_t* qs, uint16_t* d, int32_t* invalid_count,
+                        void* stream) {
+  return pack_common(TRI_TQ1, trits, N, K, scales, n_scales, qs, d, invalid_count, stream);
+}
+
+tri_status tri_unpack(int format, const uint8_t* qs, int64_t N, int64_t K, int8_t* trits,
+                      int32_t* invalid_count, void* stream) {
+  if (format != TRI_TQ2 && format != TRI_TQ1) return TRI_ERR_INVALID_ARG;
+  if (!qs || !trits) return TRI_ERR_INVALID_ARG;
+  tri_status st = check_nk(N, K);
+  if (st != TRI_OK) return st;
+  if (!aligned(trits, 16) || !aligned(qs, format == TRI_TQ2 ? 16 : 4)) return TRI_ERR_ALIGNMENT;
+  if (invalid_count && !aligned(invalid_count, 4)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  if ((st = device_info(&di)) != TRI_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (format == TRI_TQ2) return from_cuda(tri::launch_unpack_tq2(qs, N, K, trits, invalid_count, s));
+  return from_cuda(tri::launch_unpack_tq1(qs, N, K, trits, invalid_count, s));
+}
+
+int tri_gemm_auto_path(int format, int64_t M, int64_t N, int64_t K) {
+  if (format != TRI_TQ2 && format != TRI_TQ1) return -1;
+  if (M < 1 || M > kMaxDim || check_nk(N, K) != TRI_OK) return -1;
+  return auto_path(format, M, N, K);
+}
+
+size_t tri_gemm_workspace_bytes(int format, int64_t M, int64_t N, int64_t K) {
+  if (tri_gemm_auto_path(format, M, N, K) < 0) return 0;
+  DevInfo di;
+  int sms = 148;
+  if (device_info(&di) == TRI_OK) sms = di.sms;
+  size_t a = tri::gemv_mma_supported(format, M, N, K) ? tri::gemv_mma_ws_bytes(format, M, N, K, sms) : 0;
+  size_t b = tri::gemm_tc_supported(format, M, N, K) ? tri::gemm_tc_ws_bytes(format, M, N, K, sms) : 0;
+  size_t r = a > b ? a : b;
+  return r < 256 ? 256 : r;
+}
+
+tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs, const uint16_t* d,
+                    uint16_t* Y, int64_t M, int64_t N, int64_t K, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (format != TRI_TQ2 && format != TRI_TQ1) return TRI_ERR_INVALID_ARG;
+  if (path < TRI_PATH_AUTO || path > TRI_PATH_TCGEN05) return TRI_ERR_INVALID_ARG;
+  if (!X || !qs || !d || !Y) return TRI_ERR_INVALID_ARG;
+  if (M < 1 || M > kMaxDim) return TRI_ERR_SHAPE;
+  tri_status st = check_nk(N, K);
+  if (st != TRI_OK) return st;
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(d, 4)) return TRI_ERR_ALIGNMENT;
+  if (!aligned(qs, format == TRI_TQ2 ? 16 : 4)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  if ((st = device_info(&di)) != TRI_OK) return st;
+  if (path == TRI_PATH_AUTO) path = auto_path(format, M, N, K);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __half* Xh = reinterpret_cast<const __half*>(X);
+  const __half* dh = reinterpret_cast<const __half*>(d);
+  __half* Yh = reinterpret_cast<__half*>(Y);
+  switch (path) {
+    case TRI_PATH_SIMT:
+      return from_cuda(tri::launch_gemm_simt(format, Xh, qs, dh, Yh, (int)M, (int)N, (int)K, s));
+    case TRI_PATH_MMA: {
+      if (!tri::gemv_mma_supported(format, M, N, K)) return TRI_ERR_NOT_IMPLEMENTED;
+      const size_t need = tri::gemv_mma_ws_bytes(format, M, N, K, di.sms);
+      if (need && (!workspace || workspace_bytes < need)) return TRI_ERR_WORKSPACE;
+      if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
+      return from_cuda(tri::launch_gemv_mma(format, Xh, qs, dh, Yh, (int)M, (int)N, (int)K,
+                                            workspace, di.sms, s));
+    }
+    case TRI_PATH_TCGEN05: {
+      if (!tri::gemm_tc_supported(format, M, N, K)) return TRI_ERR_NOT_IMPLEMENTED;
+      const size_t need = tri::gemm_tc_ws_bytes(format, M, N, K, di.sms);
+      if (need && (!workspace || workspace_bytes < need)) return TRI_ERR_WORKSPACE;
+      if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
+      return from_cuda(tri::launch_gemm_tc(format, Xh, qs, dh, Yh, (int)M, (int)N, (int)K,
+                                           workspace, di.sms, s));
+    }
+    default:
+      return TRI_ERR_INVALID_ARG;
+  }
+}
+
+tri_status tri_gemm_tq2(const uint16_t* X, const uint8_t* qs, const uint16_t* d, uint16_t* Y,
+                        int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return tri_gemm(TRI_TQ2, TRI_PATH_AUTO, X, qs, d, Y, M, N, K, workspace, workspace_bytes, stream);
+}
+
+tri_status tri_gemm_tq1(const uint16_t* X, const uint8_t* qs, const uint16_t* d, uint16_t* Y,
+                        int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  return tri_gemm(TRI_TQ1, TRI_PATH_AUTO, X, qs, d, Y, M, N, K, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"

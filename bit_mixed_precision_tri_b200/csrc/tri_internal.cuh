@@ -1,0 +1,58 @@
+// Internal declarations shared by the library's translation units.
+// Everything here is device/host plumbing for sm_100a; the public C ABI is
+// include/tri.h.
+#pragma once
+
+#include <cstdint>
+#include <cstddef>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+
+#include "../../include/tri.h"
+
+namespace tri {
+
+constexpr int kBlock = 256;          // weights per block (one fp16 scale each)
+constexpr int kTq2BlockBytes = 64;   // 256 x 2 bits
+constexpr int kTq1BlockBytes = 52;   // 51 five-trit bytes + 1 byte for trit 255
+constexpr int kTq1Groups = 51;
+
+// ---- launchers (each returns cudaSuccess or the launch error) -------------
+cudaError_t launch_absmean(const float* W, int64_t n, float eps, float* gamma,
+                           void* ws, cudaStream_t s);
+cudaError_t launch_ternarize(const float* W, int64_t n, const float* gamma,
+                             int8_t* trits, cudaStream_t s);
+size_t absmean_ws_bytes();
+
+cudaError_t launch_pack_tq2(const int8_t* trits, int64_t N, int64_t K, const float* scales,
+                            int64_t n_scales, uint8_t* qs, uint16_t* d, int32_t* invalid,
+                            cudaStream_t s);
+cudaError_t launch_pack_tq1(const int8_t* trits, int64_t N, int64_t K, const float* scales,
+                            int64_t n_scales, uint8_t* qs, uint16_t* d, int32_t* invalid,
+                            cudaStream_t s);
+cudaError_t launch_unpack_tq2(const uint8_t* qs, int64_t N, int64_t K, int8_t* trits,
+                              int32_t* invalid, cudaStream_t s);
+cudaError_t launch_unpack_tq1(const uint8_t* qs, int64_t N, int64_t K, int8_t* trits,
+                              int32_t* invalid, cudaStream_t s);
+
+cudaError_t launch_gemm_simt(int fmt, const __half* X, const uint8_t* qs, const __half* d,
+                             __half* Y, int M, int N, int K, cudaStream_t s);
+
+// decode-regime tensor-core path (M <= 16)
+bool gemv_mma_supported(int fmt, int64_t M, int64_t N, int64_t K);
+size_t gemv_mma_ws_bytes(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const __half* d,
+                            __half* Y, int M, int N, int K, void* ws, int num_sms,
+                            cudaStream_t s);
+
+// compute-regime tcgen05 path (M >= 64)
+bool gemm_tc_supported(int fmt, int64_t M, int64_t N, int64_t K);
+size_t gemm_tc_ws_bytes(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __half* d,
+                           __half* Y, int M, int N, int K, void* ws, int num_sms,
+                           cudaStream_t s);
+
+// ---- small helpers ---------------------------------------------------------
+__host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace tri

@@ -1,0 +1,204 @@
+/*
+ * tri.h -- C ABI of the B200 ternary-weight linear-layer library (libtri_b200.so).
+ *
+ * The library implements, for NVIDIA B200 (sm_100a), the inference path of a
+ * ternary linear layer as described on the page "Scaling Laws and Efficient
+ * Inference for Ternary Language Models" (Spectra-1.1 / TriTera project page)
+ * and on "Spectra: Surprising Effectiveness of Pretraining Ternary Language
+ * Models at Scale" (section "Architecture of TriLM and FloatLM"):
+ *
+ *   absmean scale      gamma = eps + mean|W|                   ("The model", step 1)
+ *   ternarize          W_hat = round(clip(W / gamma, -1, 1))   ("The model", step 2)
+ *   TQ2 / TQ1 packing  2 bits or 1.6 bits per weight           ("Packing ternary weights")
+ *   ternary GEMM       Y = X (gamma W_hat)^T, fp32 accumulation ("The model", step 3;
+ *                      "TriRun: ternary inference on GPUs")
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Shapes: W is N x K (N output features, K input features), row-major.
+ *    X is M x K fp16 row-major, Y is M x N fp16 row-major.  K must be a
+ *    positive multiple of 256 (one block = 256 consecutive weights of a row).
+ *  - Every data pointer is a DEVICE pointer, allocated and owned by the
+ *    caller.  The library allocates nothing and never synchronizes the host;
+ *    all work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) in call order.
+ *  - fp16 tensors are passed as uint16_t bit patterns (IEEE binary16).
+ *  - Arguments are validated on the host before anything is enqueued; a
+ *    non-OK status means nothing was launched.  A launch failure reported by
+ *    the CUDA runtime returns TRI_ERR_CUDA.  No kernel traps or asserts:
+ *    data errors (non-finite weights, invalid packed codes) are reported
+ *    through device-side results described per function.
+ *  - Buffers given to one call must not overlap unless stated.
+ *
+ * Packed formats (readings of the pages, fixed by this library)
+ * -------------------------------------------------------------
+ *  TQ2 ("2 bits per weight"): the shifted digit d' = t + 1 in {0,1,2} of
+ *    weight k of a row is stored in bits 2*(k%4) .. 2*(k%4)+1 of byte k/4 of
+ *    that row, so a little-endian 32-bit word holds sixteen consecutive
+ *    weights, weight j at bits 2j ("TriRun": "each 32-bit word holds sixteen
+ *    2-bit weights").  qs is uint8[N][K/4] (64 bytes per 256-block).
+ *  TQ1 ("1.6 bits per weight"): five consecutive weights form a base-3 number
+ *    N5 = sum_j d'_j 3^(4-j) (first weight most significant), stored as the
+ *    byte floor((256*N5 + 242)/243).  Each 256-block takes 52 bytes: bytes
+ *    0..50 hold weights 5g..5g+4 of the block, byte 51 holds weight 255 as its
+ *    leading digit followed by four zero weights.  qs is uint8[N][52*K/256].
+ *  Scales (section "Fast inference on CPUs": one 16-bit scale per 256-block):
+ *    d is fp16[N][K/256]; the weight of row n, column k is d[n][k/256] * t.
+ */
+#ifndef TRI_B200_H
+#define TRI_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TRI_API __attribute__((visibility("default")))
+#else
+#define TRI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tri_status {
+    TRI_OK = 0,
+    TRI_ERR_INVALID_ARG = 1,      /* null pointer, bad enum, eps < 0 ...      */
+    TRI_ERR_SHAPE = 2,            /* M, N, K out of range or K % 256 != 0     */
+    TRI_ERR_ALIGNMENT = 3,        /* a pointer is not 16-byte aligned         */
+    TRI_ERR_NONFINITE = 4,        /* reserved for wrappers (see tri_absmean)  */
+    TRI_ERR_INVALID_CODE = 5,     /* reserved for wrappers (see tri_unpack)   */
+    TRI_ERR_CUDA = 6,             /* the CUDA runtime reported an error       */
+    TRI_ERR_NOT_IMPLEMENTED = 7,  /* the requested kernel path does not exist */
+    TRI_ERR_WORKSPACE = 8,        /* workspace null or smaller than required  */
+    TRI_ERR_NO_DEVICE = 9         /* current device is not sm_100             */
+} tri_status;
+
+typedef enum tri_format { TRI_TQ1 = 1, TRI_TQ2 = 2 } tri_format;
+
+/* Kernel choice for tri_gemm: AUTO picks by M (see tri_gemm). */
+typedef enum tri_gemm_path {
+    TRI_PATH_AUTO = 0,
+    TRI_PATH_SIMT = 1,     /* CUDA-core kernel, any M (correctness baseline)           */
+    TRI_PATH_MMA = 2,      /* decode-regime tensor-core kernel, M <= 16                */
+    TRI_PATH_TCGEN05 = 3   /* compute-regime kernel: tcgen05 MMA, TMEM accumulators    */
+} tri_gemm_path;
+
+/* Human-readable name of a status code (static string, never NULL). */
+TRI_API const char* tri_status_string(int status);
+
+/* Library ABI version (major*100 + minor). */
+TRI_API int tri_version(void);
+
+/* ------------------------------------------------------------------------
+ * Absmean scale ("The model", step 1; Spectra "Architecture": one scale per
+ * matrix, the mean absolute value of the latent weights).
+ *
+ *   gamma = RN32( RN64( RN64(S) / (N*K) ) + eps ),  S = sum |W[n][k]| exactly.
+ *
+ * The sum is formed exactly (integer accumulation per float exponent), so
+ * gamma does not depend on the order of the reduction and is bit-identical
+ * across runs and grid sizes.
+ *   W         device float32[N][K], read only.
+ *   eps       >= 0, finite (1e-6 in the pages' workloads).
+ *   gamma     device float32[1], written.  If W holds Inf or NaN, *gamma is
+ *             set to NaN (check it on the host to detect non-finite weights).
+ *   workspace device scratch of at least tri_absmean_workspace_bytes(N, K)
+ *             bytes, 16-byte aligned; its contents on entry do not matter.
+ * N*K must be below 2^40.
+ * ---------------------------------------------------------------------- */
+TRI_API size_t tri_absmean_workspace_bytes(int64_t N, int64_t K);
+TRI_API tri_status tri_absmean(const float* W, int64_t N, int64_t K, float eps, float* gamma,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Absmean ternarization ("The model", steps 1-2):
+ *   gamma as in tri_absmean, then trits[n][k] = rint(clip(W/gamma, -1, 1))
+ *   with an IEEE float32 division and round-half-to-even; a NaN quotient
+ *   (non-finite W, or gamma = 0) gives trit 0.
+ *   trits     device int8[N][K], written, values in {-1, 0, 1}.
+ * Other arguments as for tri_absmean (same workspace size).
+ * ---------------------------------------------------------------------- */
+TRI_API tri_status tri_ternarize(const float* W, int64_t N, int64_t K, float eps,
+                         int8_t* trits, float* gamma,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Packing ("Packing ternary weights": "2 bits per weight" for TQ2,
+ * "1.6 bits per weight" for TQ1; block scale per "Fast inference on CPUs").
+ *   trits     device int8[N][K] in {-1,0,1}; any other value is counted as
+ *             invalid and packed as 0.
+ *   scales    device float32, n_scales values: 1 (one scale for the matrix,
+ *             e.g. gamma from tri_ternarize) or N*K/256 (one per block,
+ *             row-major [N][K/256]).  d = fp16(scale), round to nearest even.
+ *   qs        device uint8: N*K/4 bytes (TQ2) or N*(K/256)*52 bytes (TQ1).
+ *   d         device fp16[N][K/256], written.
+ *   invalid_count  device int32[1] or NULL; set to the number of invalid
+ *             input trits.
+ * qs must be 16-byte aligned for TQ2 and 4-byte aligned for TQ1; d 4-byte.
+ * ---------------------------------------------------------------------- */
+TRI_API tri_status tri_pack_tq2(const int8_t* trits, int64_t N, int64_t K,
+                        const float* scales, int64_t n_scales,
+                        uint8_t* qs, uint16_t* d, int32_t* invalid_count, void* stream);
+TRI_API tri_status tri_pack_tq1(const int8_t* trits, int64_t N, int64_t K,
+                        const float* scales, int64_t n_scales,
+                        uint8_t* qs, uint16_t* d, int32_t* invalid_count, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Unpacking ("2 bits per weight": d' = (b >> 2j) & 3; "1.6 bits per weight":
+ * the multiply-by-3 / high-byte digit extraction).
+ *   format    TRI_TQ2 or TRI_TQ1.
+ *   qs        packed plane as written by tri_pack_*.
+ *   trits     device int8[N][K], written.
+ *   invalid_count  device int32[1] or NULL; set to the number of invalid
+ *             codes: TQ2 fields equal to 3; TQ1 bytes outside the encoder's
+ *             243-value image, plus block-final bytes whose four padding
+ *             digits are not the zero weight.  Invalid codes are still decoded
+ *             by the same rule (t = d' - 1, so a TQ2 field of 3 gives 2), so
+ *             the output is defined for every input byte.
+ * ---------------------------------------------------------------------- */
+TRI_API tri_status tri_unpack(int format, const uint8_t* qs, int64_t N, int64_t K,
+                      int8_t* trits, int32_t* invalid_count, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Ternary GEMM ("The model", step 3: Y = X (gamma W_hat)^T; "TriRun": fp16
+ * activations, fp32 accumulation, fp16 output):
+ *
+ *   Y[m][n] = fp16_RN( sum_b d[n][b] * sum_{k in block b} X[m][k] * t[n][k] )
+ *
+ * accumulated in float32 (the summation order is the kernel's; results are
+ * deterministic for a given device, path and shape).
+ *   X         device fp16[M][K], 16-byte aligned.
+ *   qs, d     packed weights in `format`, as written by tri_pack_*; qs
+ *             16-byte aligned (TQ2) or 4-byte aligned (TQ1).  Codes that
+ *             are invalid give unspecified (but finite, non-faulting) output.
+ *   Y         device fp16[M][N], 16-byte aligned, written.
+ *   M >= 1, N >= 1, K >= 256 with K % 256 == 0; M, N, K < 2^31.
+ *   workspace device scratch of at least tri_gemm_workspace_bytes(format, M,
+ *             N, K) bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE
+ *             (the kernels leave it zeroed for the next call).  Calls that
+ *             share one workspace must be ordered (same stream, or events).
+ *   path      TRI_PATH_AUTO chooses TRI_PATH_MMA for M <= 16 and
+ *             TRI_PATH_TCGEN05 for M >= 64 (TQ2; TQ1 for M >= 64 too), else
+ *             the best available; an explicit path that cannot serve the
+ *             shape returns TRI_ERR_NOT_IMPLEMENTED.
+ * ---------------------------------------------------------------------- */
+TRI_API size_t tri_gemm_workspace_bytes(int format, int64_t M, int64_t N, int64_t K);
+TRI_API tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs,
+                    const uint16_t* d, uint16_t* Y, int64_t M, int64_t N, int64_t K,
+                    void* workspace, size_t workspace_bytes, void* stream);
+TRI_API tri_status tri_gemm_tq2(const uint16_t* X, const uint8_t* qs, const uint16_t* d,
+                        uint16_t* Y, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, void* stream);
+TRI_API tri_status tri_gemm_tq1(const uint16_t* X, const uint8_t* qs, const uint16_t* d,
+                        uint16_t* Y, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Kernel that tri_gemm would launch for this call under TRI_PATH_AUTO
+ * (one of tri_gemm_path), or -1 if the shape is invalid. */
+TRI_API int tri_gemm_auto_path(int format, int64_t M, int64_t N, int64_t K);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TRI_B200_H */

@@ -23,7 +23,8 @@ Readings of points the pages leave open:
 
 R1  gamma is computed from the EXACT sum S = sum|W| (order independent):
     mean = RN64(RN64(S) / (N*K)), gamma = RN32(RN64(mean + eps)).
-R2  W/gamma is an IEEE float32 division; clip to [-1, 1]; round half to even.
+R2  W/gamma is an IEEE float32 division; clip to [-1, 1]; round half to even;
+    a NaN quotient (non-finite W, or gamma = 0) gives trit 0.
 R3  TQ2 byte i of a row holds trits 4i..4i+3, trit 4i+j in bits 2j..2j+1, so a
     little-endian 32-bit word holds sixteen trits, trit j at bits 2j.
     Storage is two planes: qs (64 B per 256-block) and d (one fp16 per block).
@@ -94,7 +95,9 @@ def absmean_gamma(W: np.ndarray, eps: float) -> np.float32:
 def ternarize(W: np.ndarray, gamma) -> np.ndarray:
     """trits = round(clip(W / gamma, -1, 1)) in {-1, 0, 1}, reading R2."""
     a = np.ascontiguousarray(W, dtype=np.float32)
-    x = a / np.float32(gamma)                 # float32 / float32, IEEE RN
+    with np.errstate(divide="ignore", invalid="ignore"):
+        x = a / np.float32(gamma)             # float32 / float32, IEEE RN
+    x = np.where(np.isnan(x), np.float32(0.0), x)   # NaN quotient -> trit 0 (R2)
     x = np.clip(x, np.float32(-1.0), np.float32(1.0))
     return np.rint(x).astype(np.int8)         # rint: half to even
 
@@ -120,9 +123,20 @@ def block_scales_fp16(scales, N: int, K: int) -> np.ndarray:
 # --------------------------------------------------------------------------
 # a3: TQ2 pack / unpack  [TLS "2 bits per weight"; TriRun storage line]
 # --------------------------------------------------------------------------
+def invalid_trit_count(trits) -> int:
+    """Number of input values outside {-1, 0, 1} (packed as 0, reading R7)."""
+    t = np.asarray(trits, dtype=np.int64)
+    return int(np.count_nonzero((t < -1) | (t > 1)))
+
+
+def _valid_trits(trits) -> np.ndarray:
+    t = np.asarray(trits, dtype=np.int64)
+    return np.where((t < -1) | (t > 1), 0, t)
+
+
 def pack_tq2(trits: np.ndarray, scales):
     """Return (qs uint8[N][K/4], d fp16[N][K/256]); reading R3."""
-    t = np.asarray(trits, dtype=np.int64)
+    t = _valid_trits(trits)
     N, K = t.shape
     assert K % BLOCK == 0
     dp = (t + 1).reshape(N, K // 4, 4)                 # d' = d + 1 in {0,1,2}
@@ -171,7 +185,7 @@ def encode_kp(n: int, k: int, p: int) -> int:
 
 def pack_tq1(trits: np.ndarray, scales):
     """Return (qs uint8[N][(K/256)*52], d fp16[N][K/256]); readings R4, R5."""
-    t = np.asarray(trits, dtype=np.int64)
+    t = _valid_trits(trits)
     N, K = t.shape
     assert K % BLOCK == 0
     nb = K // BLOCK

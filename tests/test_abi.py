@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function declared in include/tri.h, and rejects bad arguments before
+touching the device (nothing here launches a kernel)."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from bit_mixed_precision_tri_b200 import _lib
+
+FAKE = 1 << 20        # a non-null, 256-byte-aligned address that is never dereferenced
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(_lib.LIB_PATH):
+        from bit_mixed_precision_tri_b200 import build
+        build.build()
+    return _lib.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _lib.declared_symbols()
+    assert len(declared) >= 13
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in declared:
+        assert name in exported, name
+        assert hasattr(L, name)
+    assert set(_lib.SIGNATURES) == set(declared)
+
+
+def test_status_strings_and_version(L):
+    assert L.tri_version() >= 100
+    for s in range(10):
+        assert L.tri_status_string(s)
+    assert L.tri_status_string(12345) == b"unknown status"
+
+
+def test_gemm_argument_validation(L):
+    g = L.tri_gemm
+    ok = dict(fmt=2, path=0, X=FAKE, qs=FAKE, d=FAKE, Y=FAKE, M=1, N=8, K=256)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["fmt"], a["path"], a["X"], a["qs"], a["d"], a["Y"], a["M"], a["N"], a["K"],
+                 None, 0, None)
+
+    assert call(fmt=3) == 1
+    assert call(path=9) == 1
+    assert call(X=None) == 1
+    assert call(M=0) == 2
+    assert call(N=0) == 2
+    assert call(K=255) == 2
+    assert call(K=300) == 2
+    assert call(K=0) == 2
+    assert call(M=1 << 31) == 2
+    assert call(X=FAKE + 8) == 3
+    assert call(Y=FAKE + 2) == 3
+    assert call(qs=FAKE + 4) == 3                   # TQ2 planes need 16-byte alignment
+    assert call(fmt=1, qs=FAKE + 4, X=FAKE + 8) == 3  # X still misaligned
+
+
+def test_pack_unpack_and_absmean_validation(L):
+    assert L.tri_pack_tq2(None, 4, 256, FAKE, 1, FAKE, FAKE, None, None) == 1
+    assert L.tri_pack_tq2(FAKE, 4, 256, FAKE, 3, FAKE, FAKE, None, None) == 1   # n_scales
+    assert L.tri_pack_tq1(FAKE, 4, 100, FAKE, 1, FAKE, FAKE, None, None) == 2
+    assert L.tri_pack_tq2(FAKE + 1, 4, 256, FAKE, 1, FAKE, FAKE, None, None) == 3
+    assert L.tri_unpack(7, FAKE, 4, 256, FAKE, None, None) == 1
+    assert L.tri_unpack(2, FAKE, 4, 512 + 1, FAKE, None, None) == 2
+    ws = L.tri_absmean_workspace_bytes(4, 256)
+    assert ws >= 256 * 8
+    assert L.tri_absmean(FAKE, 4, 256, -1.0, FAKE, FAKE, ws, None) == 1          # eps < 0
+    assert L.tri_absmean(FAKE, 4, 256, 1e-6, FAKE, FAKE, ws - 1, None) == 8      # workspace
+    assert L.tri_absmean(FAKE, 4, 256, 1e-6, FAKE, None, ws, None) == 8
+    assert L.tri_ternarize(FAKE, 4, 256, 1e-6, None, FAKE, FAKE, ws, None) == 1
+
+
+def test_auto_path_and_workspace_query(L):
+    assert L.tri_gemm_auto_path(2, 0, 8, 256) == -1
+    assert L.tri_gemm_auto_path(5, 1, 8, 256) == -1
+    for fmt in (1, 2):
+        for M in (1, 16, 64, 256):
+            p = L.tri_gemm_auto_path(fmt, M, 4096, 4096)
+            assert p in (1, 2, 3)
+            assert L.tri_gemm_workspace_bytes(fmt, M, 4096, 4096) >= 256

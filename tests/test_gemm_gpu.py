@@ -1,0 +1,154 @@
+"""GPU parity of the ternary GEMM against the FP64 CPU oracle, for every
+kernel path, through the C ABI.  Bar (from the workload statement):
+|y - y_ref| <= 1e-3 * gamma_n * sum_k |x_mk| + 2^-10 * |y_ref|, gamma_n the
+largest block scale of output row n."""
+import numpy as np
+import pytest
+import torch
+
+import bit_mixed_precision_tri_b200 as tri
+from bit_mixed_precision_tri_b200 import inputs
+from oracle import tri_oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+PATHS = {"simt": tri.PATH_SIMT, "mma": tri.PATH_MMA, "tcgen05": tri.PATH_TCGEN05}
+
+
+def _supported(path, fmt, M, N, K):
+    """Whether an explicit path serves this shape (the library answers)."""
+    if path == tri.PATH_SIMT:
+        return True
+    X = torch.zeros(M, K, dtype=torch.float16, device=DEV)
+    qs = torch.zeros(N, tri.packed_row_bytes(fmt, K), dtype=torch.uint8, device=DEV)
+    d = torch.zeros(N, K // 256, dtype=torch.float16, device=DEV)
+    try:
+        tri.gemm(X, qs, d, N, K, fmt, path=path)
+        return True
+    except tri.TriError as e:
+        if e.status == 7:
+            return False
+        raise
+
+
+def _check(Y, X, trits, d, rows=None):
+    y_ref = O.gemm_f64(X, trits, d)
+    y = Y.float().cpu().numpy().astype(np.float64)
+    if rows is not None:
+        y = y[:, rows]
+    tol = O.gemm_tolerance(X, d, y_ref)
+    err = np.abs(y - y_ref)
+    bad = err > tol
+    assert not bad.any(), f"{bad.sum()} outputs out of tolerance; worst {(err - tol).max()}"
+    assert np.all(np.isfinite(y))
+
+
+def _case(M, N, K, seed, fmt, per_block=False, p_zero=None):
+    if p_zero is None:
+        W = inputs.latent_weights(N, K, seed)
+        trits, g = O.absmean_ternarize(W.numpy(), 1e-6)
+        scales = np.array([g], np.float32)
+    else:
+        trits = inputs.random_trits(N, K, p_zero, seed).numpy()
+        scales = inputs.block_scales(N, K, seed + 1).numpy() if per_block else np.array([0.03], np.float32)
+    qs, d = O.pack(fmt, trits, scales)
+    X = inputs.activations(M, K, seed + 100).numpy()
+    return X, trits, qs, d
+
+
+SMALL = [(1, 256, 1024), (1, 1, 256), (2, 37, 768), (3, 300, 1024), (5, 1000, 512), (8, 64, 2048),
+         (13, 129, 768), (16, 256, 4096), (16, 17, 256)]
+MID = [(33, 256, 1024), (64, 256, 512), (100, 384, 768), (128, 512, 1024), (200, 640, 2048)]
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+@pytest.mark.parametrize("pname", list(PATHS))
+@pytest.mark.parametrize("M,N,K", SMALL + MID)
+def test_gemm_paths_vs_oracle(fmt, pname, M, N, K):
+    path = PATHS[pname]
+    if not _supported(path, fmt, M, N, K):
+        pytest.skip(f"{pname} does not serve {fmt} M={M} N={N} K={K}")
+    X, trits, qs, d = _case(M, N, K, 1000 + 7 * M + N, fmt)
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, fmt, path=path)
+    _check(Y, X, trits, d)
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+@pytest.mark.parametrize("M", [1, 16, 128])
+@pytest.mark.parametrize("p_zero", [0.3, 0.9])
+def test_gemm_per_block_scales_and_sparsity(fmt, M, p_zero):
+    N, K = 512, 4096
+    X, trits, qs, d = _case(M, N, K, 20 + int(10 * p_zero), fmt, per_block=True, p_zero=p_zero)
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, fmt)
+    _check(Y, X, trits, d)
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+def test_gemm_special_cases(fmt):
+    M, N, K = 4, 96, 1024
+    X = inputs.activations(M, K, 5).numpy()
+    Xd = torch.from_numpy(X).to(DEV)
+    for pname, path in PATHS.items():
+        if not _supported(path, fmt, M, N, K):
+            continue
+        for kind in ("zero", "ones", "single"):
+            trits = np.zeros((N, K), np.int8)
+            if kind == "ones":
+                trits[:] = 1
+            elif kind == "single":
+                trits[5, 700] = -1
+            qs, d = O.pack(fmt, trits, np.float32(0.0234))
+            Y = tri.gemm(Xd, torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV), N, K, fmt,
+                         path=path)
+            _check(Y, X, trits, d)
+            if kind == "single" and path == tri.PATH_SIMT:
+                y = Y.float().cpu().numpy()
+                exp = (-np.float64(d[5, 2]) * X[:, 700].astype(np.float64)).astype(np.float16)
+                assert np.array_equal(y[:, 5].astype(np.float16), exp)
+                assert np.all(np.delete(y, 5, axis=1) == 0)
+
+
+def test_gemm_tiny_config_all_formats():
+    """Tiny correctness case: W 256x1024 ~ N(0, 0.02) seed 0, X 1x1024 seed 1."""
+    W = inputs.latent_weights(256, 1024, 0)
+    X = inputs.activations(1, 1024, 1)
+    for fmt in ("tq2", "tq1"):
+        layer = tri.TernaryLinear.from_latent(W.to(DEV), fmt)
+        Y = layer(X.to(DEV))
+        t_ref, g_ref = O.absmean_ternarize(W.numpy(), 1e-6)
+        _, d_ref = O.pack(fmt, t_ref, np.array([g_ref], np.float32))
+        assert np.array_equal(layer.d.cpu().numpy().view(np.uint16), d_ref.view(np.uint16))
+        _check(Y, X.numpy(), t_ref, d_ref)
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+@pytest.mark.parametrize("M", [1, 16, 256])
+def test_gemm_full_size_sampled(fmt, M):
+    """Largest layer shape (8192 x 28672): sampled output rows against the oracle,
+    in the launch configuration the bench uses (AUTO path)."""
+    N, K = 8192, 28672
+    trits = inputs.random_trits(N, K, 0.31, 77)
+    scale = torch.tensor([0.0159], dtype=torch.float32)
+    qs, d = tri.pack(trits.to(DEV), scale.to(DEV), fmt)
+    X = inputs.activations(M, K, 78)
+    Y = tri.gemm(X.to(DEV), qs, d, N, K, fmt)
+    rows = np.sort(np.random.default_rng(M).choice(N, 48, replace=False))
+    rows[0], rows[-1] = 0, N - 1
+    t_rows = trits.numpy()[rows]
+    _, d_rows = O.pack(fmt, t_rows, scale.numpy())
+    y_ref = O.gemm_f64(X.numpy(), t_rows, d_rows)
+    y = Y.float().cpu().numpy()[:, rows].astype(np.float64)
+    tol = O.gemm_tolerance(X.numpy(), d_rows, y_ref)
+    assert np.all(np.abs(y - y_ref) <= tol)
+
+
+def test_gemm_repeat_deterministic():
+    M, N, K = 8, 4096, 4096
+    X, trits, qs, d = _case(M, N, K, 4, "tq2")
+    args = (torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV),
+            N, K, "tq2")
+    Y1 = tri.gemm(*args)
+    Y2 = tri.gemm(*args)
+    assert torch.equal(Y1, Y2)
