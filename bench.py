@@ -307,6 +307,57 @@ def run_ours(args, rank, world, device):
     return res
 
 
+# ------------------------------------------------------------------ other rows
+def measure_rows(device, N=28672, K=8192, reps=5):
+    """Time the offline rows of the path (absmean, ternarize, pack, unpack) on
+    the largest weight of the 70B-like block (inputs larger than L2), with
+    CUDA events; algorithmic bytes per element are stated per row."""
+    import bit_mixed_precision_tri_b200 as tri
+    from bit_mixed_precision_tri_b200 import inputs
+    n = N * K
+    W = inputs.latent_weights(N, K, 12).to(device)
+    L = tri._lib.lib()
+    ws = torch.zeros(L.tri_absmean_workspace_bytes(N, K), dtype=torch.uint8, device=device)
+    g = torch.empty(1, dtype=torch.float32, device=device)
+    trits = torch.empty(N, K, dtype=torch.int8, device=device)
+    q2 = torch.empty(N, K // 4, dtype=torch.uint8, device=device)
+    q1 = torch.empty(N, (K // 256) * 52, dtype=torch.uint8, device=device)
+    dd = torch.empty(N, K // 256, dtype=torch.float16, device=device)
+    out = torch.empty(N, K, dtype=torch.int8, device=device)
+    st = torch.cuda.current_stream(device).cuda_stream
+    P = lambda t: t.data_ptr()
+    ops = {
+        "absmean": (lambda: L.tri_absmean(P(W), N, K, 1e-6, P(g), P(ws), ws.numel(), st), 4.0),
+        "ternarize": (lambda: L.tri_ternarize(P(W), N, K, 1e-6, P(trits), P(g), P(ws), ws.numel(), st),
+                      9.0),
+        "pack_tq2": (lambda: L.tri_pack_tq2(P(trits), N, K, P(g), 1, P(q2), P(dd), None, st),
+                     1.0 + 0.25 + 2 / 256),
+        "pack_tq1": (lambda: L.tri_pack_tq1(P(trits), N, K, P(g), 1, P(q1), P(dd), None, st),
+                     1.0 + 52 / 256 + 2 / 256),
+        "unpack_tq2": (lambda: L.tri_unpack(2, P(q2), N, K, P(out), None, st), 0.25 + 1.0),
+        "unpack_tq1": (lambda: L.tri_unpack(1, P(q1), N, K, P(out), None, st), 52 / 256 + 1.0),
+    }
+    res = {}
+    for name, (fn, bpe) in ops.items():
+        for _ in range(2):
+            assert fn() == 0, name
+        times = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            assert fn() == 0, name
+            b.record()
+            torch.cuda.synchronize(device)
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        res[name] = {"us": round(ms * 1e3, 1), "GB/s": round(n * bpe / (ms * 1e-3) / 1e9, 1),
+                     "bytes_per_weight": round(bpe, 4)}
+    res["shape"] = f"{N}x{K}"
+    del W, trits, q2, q1, dd, out
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ oracle arm
 def oracle_sample(w, budget_s=12.0):
     """Time the CPU oracle (as it stands) on a bounded sample of the workload:
@@ -396,6 +447,7 @@ def main():
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--fmt", default=None, choices=[None, "tq2", "tq1"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip timing the offline rows")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -417,6 +469,8 @@ def main():
                                              device_id=device)
     try:
         res = run_ours(args, rank, world, device)
+        if not args.no_rows:
+            res["rows"] = measure_rows(device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             w = workload_from_args(args.workload, args.M, args.fmt)
             v, unit, desc, threads = oracle_sample(w, budget_s=10.0)

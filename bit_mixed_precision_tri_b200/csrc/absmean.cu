@@ -38,13 +38,21 @@ __device__ __forceinline__ float4 ld_stream_f4(const float4* p) {
   return v;
 }
 
-__device__ __forceinline__ void bin_add(unsigned long long* wbins, float x, unsigned& bad) {
+// Add |x| to the warp's exponent bins.  Lanes holding the same exponent are
+// grouped with match.any, their 24-bit mantissas summed with redux.sync
+// (< 2^29, exact in 32 bits), and one lane per group issues the atomic, so a
+// warp step costs one shared atomic per distinct exponent instead of 32.
+// All 32 lanes must call this together.
+__device__ __forceinline__ void bin_add_warp(unsigned long long* wbins, float x, unsigned& bad) {
   const unsigned u = __float_as_uint(x) & 0x7FFFFFFFu;
-  const unsigned e = u >> 23;
-  if (e == 255u) { bad = 1u; return; }
-  if (u == 0u) return;
-  const unsigned m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-  atomicAdd(&wbins[e ? e : 1u], (unsigned long long)m);
+  unsigned e = u >> 23;
+  unsigned m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+  if (e == 255u) { bad = 1u; m = 0u; }
+  if (e == 0u) e = 1u;
+  const unsigned grp = __match_any_sync(0xFFFFFFFFu, e);
+  const unsigned sum = __reduce_add_sync(grp, m);
+  if ((threadIdx.x & 31) == (unsigned)(__ffs(grp) - 1) && sum != 0u)
+    atomicAdd(&wbins[e], (unsigned long long)sum);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -57,15 +65,20 @@ absmean_bins_kernel(const float* __restrict__ W, int64_t n, AbsmeanWs* ws) {
   const int64_t n4 = n >> 2;
   const float4* W4 = reinterpret_cast<const float4*>(W);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n4; i += stride) {
-    const float4 v = ld_stream_f4(W4 + i);
-    bin_add(wb, v.x, bad);
-    bin_add(wb, v.y, bad);
-    bin_add(wb, v.z, bad);
-    bin_add(wb, v.w, bad);
+  // whole warps iterate together (the bins update is a warp collective)
+  for (int64_t base = (int64_t)blockIdx.x * kThreads; base < n4; base += stride) {
+    const int64_t i = base + threadIdx.x;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < n4) v = ld_stream_f4(W4 + i);
+    bin_add_warp(wb, v.x, bad);
+    bin_add_warp(wb, v.y, bad);
+    bin_add_warp(wb, v.z, bad);
+    bin_add_warp(wb, v.w, bad);
   }
-  for (int64_t i = (n4 << 2) + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride)
-    bin_add(wb, W[i], bad);
+  for (int64_t base = (n4 << 2) + (int64_t)blockIdx.x * kThreads; base < n; base += stride) {
+    const int64_t i = base + threadIdx.x;
+    bin_add_warp(wb, i < n ? W[i] : 0.f, bad);
+  }
   const int any_bad = __syncthreads_or((int)bad);
   for (int b = threadIdx.x; b < kBins; b += kThreads) {
     unsigned long long s = 0ull;
@@ -76,15 +89,23 @@ absmean_bins_kernel(const float* __restrict__ W, int64_t n, AbsmeanWs* ws) {
   if (threadIdx.x == 0 && any_bad) atomicOr(&ws->nonfinite, 1u);
 }
 
-// bits [lo, lo+cnt) of a little-endian multi-limb integer (cnt <= 64)
-__device__ unsigned long long limb_bits(const unsigned* L, int nl, int lo, int cnt) {
-  unsigned long long r = 0ull;
-  for (int i = 0; i < cnt; ++i) {
-    const int b = lo + i;
-    if (b < 0 || (b >> 5) >= nl) continue;
-    r |= (unsigned long long)((L[b >> 5] >> (b & 31)) & 1u) << i;
-  }
-  return r;
+// 64 bits of a little-endian multi-limb integer starting at bit `pos` (pos >= 0)
+__device__ unsigned long long limb_window(const unsigned* L, int nl, int pos) {
+  const int w = pos >> 5, off = pos & 31;
+  unsigned long long lo = 0ull, mid = 0ull, hi = 0ull;
+  if (w < nl) lo = L[w];
+  if (w + 1 < nl) mid = L[w + 1];
+  if (w + 2 < nl) hi = L[w + 2];
+  const unsigned long long v = lo | (mid << 32);
+  return off ? ((v >> off) | (hi << (64 - off))) : v;
+}
+
+// true if any bit below `pos` is set
+__device__ bool limb_any_below(const unsigned* L, int pos) {
+  const int w = pos >> 5, off = pos & 31;
+  for (int i = 0; i < w; ++i)
+    if (L[i]) return true;
+  return off && (L[w] & ((1u << off) - 1u));
 }
 
 __global__ void absmean_finalize_kernel(AbsmeanWs* ws, int64_t n, float eps, float* gamma) {
@@ -118,14 +139,13 @@ __global__ void absmean_finalize_kernel(AbsmeanWs* ws, int64_t n, float eps, flo
   double s64 = 0.0;
   if (top >= 0) {
     if (top <= 52) {
-      s64 = ldexp((double)limb_bits(L, NL, 0, top + 1), -149);
+      s64 = ldexp((double)limb_window(L, NL, 0), -149);   // exact: fits in 53 bits
     } else {
       const int sh = top - 52;
-      unsigned long long mant = limb_bits(L, NL, sh, 53);
-      const unsigned rbit = (unsigned)limb_bits(L, NL, sh - 1, 1);
-      bool sticky = false;
-      for (int b = 0; b < sh - 1 && !sticky; ++b) sticky = limb_bits(L, NL, b, 1) != 0ull;
-      if (rbit && (sticky || (mant & 1ull))) ++mant;   // round half to even
+      unsigned long long mant = limb_window(L, NL, sh) & ((1ull << 53) - 1ull);
+      const bool rbit = (limb_window(L, NL, sh - 1) & 1ull) != 0ull;
+      const bool sticky = limb_any_below(L, sh - 1);
+      if (rbit && (sticky || (mant & 1ull))) ++mant;     // round half to even
       s64 = ldexp((double)mant, sh - 149);
     }
   }

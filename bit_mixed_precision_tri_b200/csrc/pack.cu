@@ -53,8 +53,8 @@ pack_tq2_kernel(const int8_t* __restrict__ trits, int64_t nwords, uint32_t* __re
                 int32_t* invalid) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  int bad = 0;
   for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nwords; base += stride, i += stride) {
-    int bad = 0;
     if (i < nwords) {
       const uint4 v = reinterpret_cast<const uint4*>(trits)[i];
       const unsigned w4[4] = {v.x, v.y, v.z, v.w};
@@ -68,8 +68,8 @@ pack_tq2_kernel(const int8_t* __restrict__ trits, int64_t nwords, uint32_t* __re
         }
       qs[i] = word;
     }
-    block_count_add(bad, invalid);
   }
+  block_count_add(bad, invalid);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -79,8 +79,8 @@ pack_tq1_kernel(const int8_t* __restrict__ trits, int64_t N, int64_t K, uint8_t*
   const int64_t nbytes = N * nb * kTq1BlockBytes;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  int bad = 0;
   for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nbytes; base += stride, i += stride) {
-    int bad = 0;
     if (i < nbytes) {
       const int64_t rowblk = i / kTq1BlockBytes;          // n * nb + b
       const int j = (int)(i - rowblk * kTq1BlockBytes);
@@ -97,8 +97,8 @@ pack_tq1_kernel(const int8_t* __restrict__ trits, int64_t N, int64_t K, uint8_t*
       }
       qs[i] = (uint8_t)((n5 * 256u + 242u) / 243u);
     }
-    block_count_add(bad, invalid);
   }
+  block_count_add(bad, invalid);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -114,8 +114,8 @@ unpack_tq2_kernel(const uint32_t* __restrict__ qs, int64_t nwords, int8_t* __res
                   int32_t* invalid) {
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  int bad = 0;
   for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nwords; base += stride, i += stride) {
-    int bad = 0;
     if (i < nwords) {
       const unsigned w = qs[i];
       unsigned out[4];
@@ -132,8 +132,8 @@ unpack_tq2_kernel(const uint32_t* __restrict__ qs, int64_t nwords, int8_t* __res
       }
       reinterpret_cast<uint4*>(trits)[i] = make_uint4(out[0], out[1], out[2], out[3]);
     }
-    block_count_add(bad, invalid);
   }
+  block_count_add(bad, invalid);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -143,8 +143,8 @@ unpack_tq1_kernel(const uint8_t* __restrict__ qs, int64_t N, int64_t K, int8_t* 
   const int64_t nbytes = N * nb * kTq1BlockBytes;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  int bad = 0;
   for (int64_t base = (int64_t)blockIdx.x * kThreads; base < nbytes; base += stride, i += stride) {
-    int bad = 0;
     if (i < nbytes) {
       const int64_t rowblk = i / kTq1BlockBytes;
       const int j = (int)(i - rowblk * kTq1BlockBytes);
@@ -170,8 +170,8 @@ unpack_tq1_kernel(const uint8_t* __restrict__ qs, int64_t N, int64_t K, int8_t* 
                ((n5 * 256u + 242u) / 243u) == byte;
       }
     }
-    block_count_add(bad, invalid);
   }
+  block_count_add(bad, invalid);
 }
 
 }  // namespace
