@@ -32,6 +32,8 @@
 //  * Partial sums of a row tile split across CTAs are combined by the last
 //    CTA to finish (an atomic ticket, no waiting), in CTA order, so results
 //    are deterministic.
+#include <mutex>
+
 #include <cudaTypedefs.h>
 
 #include "sm100_ptx.cuh"
@@ -496,6 +498,62 @@ cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const _
   if (!gemv_mma_supported(fmt, M, N, K)) return cudaErrorNotSupported;
   if (M <= 8) return launch_mp<8>(X, qs, d, Y, M, N, K, ws, num_sms, s);
   return launch_mp<16>(X, qs, d, Y, M, N, K, ws, num_sms, s);
+}
+
+// ---------------------------------------------------------------------------
+// Static-scratch variant for callers that cannot allocate device memory.
+//
+// Some hosts of this library may not call cudaMalloc at all: a plugin inside
+// a framework that owns every device allocation, code that runs while a CUDA
+// graph is being captured (where an allocation would be recorded into, or
+// break, the capture), or a real-time loop that has to keep a fixed memory
+// footprint.  They still pass X, the packed weights and Y, but the scratch
+// this kernel needs (prepared activations, split-K partials, tickets) lives
+// in the file-scope array below instead of a caller-provided workspace.
+//
+// The array is a module global: every device that loads the library keeps
+// kNoAllocScratchBytes reserved until the process exits, and every call on a
+// device uses the same bytes, so calls that can overlap on that device (two
+// streams, or two host threads) race and must be ordered by the caller.
+// Host code only ever sees a host-side stand-in for the symbol; the device
+// address is looked up with cudaGetSymbolAddress once per device, with that
+// device current, on the first call there (which may also load the module, so
+// make that first call before any stream capture).
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDev = 64;
+void* g_scratch_addr[kMaxDev];
+cudaError_t g_scratch_err[kMaxDev];
+std::once_flag g_scratch_once[kMaxDev];
+}  // namespace
+
+size_t gemv_noalloc_scratch_limit() { return kNoAllocScratchBytes; }
+
+size_t gemv_noalloc_scratch_need(int64_t M, int64_t N, int64_t K, int num_sms) {
+  return layout_for(M, N, K, num_sms).total;
+}
+
+cudaError_t launch_gemv_mma_noalloc(const __half* X, const uint8_t* qs, const __half* d, __half* Y,
+                                    int M, int N, int K, int num_sms, cudaStream_t s) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  std::call_once(g_scratch_once[dev], [dev]() {
+    void* ptr = nullptr;
+    g_scratch_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    g_scratch_addr[dev] = ptr;
+  });
+  if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
+  const Layout L = layout_for(M, N, K, num_sms);
+  if (L.total > kNoAllocScratchBytes) return cudaErrorInvalidValue;
+  uint8_t* ws = static_cast<uint8_t*>(g_scratch_addr[dev]);
+  // the tickets must start at zero; the array keeps whatever the last call left
+  e = cudaMemsetAsync(ws + L.off_cnt, 0, L.off_xil - L.off_cnt, s);
+  if (e != cudaSuccess) return e;
+  return launch_gemv_mma(TRI_TQ2, X, qs, d, Y, M, N, K, ws, num_sms, s);
 }
 
 }  // namespace tri

@@ -77,6 +77,7 @@ const char* tri_status_string(int status) {
     case TRI_ERR_NOT_IMPLEMENTED: return "kernel path not available for this shape";
     case TRI_ERR_WORKSPACE: return "workspace missing or too small";
     case TRI_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    case TRI_ERR_SCRATCH_LIMIT: return "shape needs more scratch than the no-alloc entry point's static 8 MiB array";
     default: return "unknown status";
   }
 }
@@ -210,6 +211,29 @@ tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs, 
     default:
       return TRI_ERR_INVALID_ARG;
   }
+}
+
+int tri_gemm_tq2_noalloc_fits(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || M > 16 || check_nk(N, K) != TRI_OK) return 0;
+  DevInfo di;
+  if (device_info(&di) != TRI_OK) return 0;
+  return tri::gemv_noalloc_scratch_need(M, N, K, di.sms) <= tri::gemv_noalloc_scratch_limit() ? 1 : 0;
+}
+
+tri_status tri_gemm_tq2_noalloc(const uint16_t* X, const uint8_t* qs, const uint16_t* d, uint16_t* Y,
+                                int64_t M, int64_t N, int64_t K, void* stream) {
+  if (!X || !qs || !d || !Y) return TRI_ERR_INVALID_ARG;
+  if (M < 1 || M > 16) return TRI_ERR_SHAPE;
+  tri_status st = check_nk(N, K);
+  if (st != TRI_OK) return st;
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(d, 4) || !aligned(qs, 16)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  if ((st = device_info(&di)) != TRI_OK) return st;
+  if (tri::gemv_noalloc_scratch_need(M, N, K, di.sms) > tri::gemv_noalloc_scratch_limit())
+    return TRI_ERR_SCRATCH_LIMIT;
+  return from_cuda(tri::launch_gemv_mma_noalloc(
+      reinterpret_cast<const __half*>(X), qs, reinterpret_cast<const __half*>(d),
+      reinterpret_cast<__half*>(Y), (int)M, (int)N, (int)K, di.sms, static_cast<cudaStream_t>(stream)));
 }
 
 tri_status tri_gemm_tq2(const uint16_t* X, const uint8_t* qs, const uint16_t* d, uint16_t* Y,

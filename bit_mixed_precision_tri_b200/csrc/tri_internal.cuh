@@ -45,6 +45,12 @@ cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const _
                             __half* Y, int M, int N, int K, void* ws, int num_sms,
                             cudaStream_t s);
 
+// decode-regime path with library-owned static scratch (no allocation)
+size_t gemv_noalloc_scratch_limit();
+size_t gemv_noalloc_scratch_need(int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv_mma_noalloc(const __half* X, const uint8_t* qs, const __half* d, __half* Y,
+                                    int M, int N, int K, int num_sms, cudaStream_t s);
+
 // compute-regime tcgen05 path (M >= 64)
 bool gemm_tc_supported(int fmt, int64_t M, int64_t N, int64_t K);
 size_t gemm_tc_ws_bytes(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);

@@ -71,7 +71,8 @@ typedef enum tri_status {
     TRI_ERR_CUDA = 6,             /* the CUDA runtime reported an error       */
     TRI_ERR_NOT_IMPLEMENTED = 7,  /* the requested kernel path does not exist */
     TRI_ERR_WORKSPACE = 8,        /* workspace null or smaller than required  */
-    TRI_ERR_NO_DEVICE = 9         /* current device is not sm_100             */
+    TRI_ERR_NO_DEVICE = 9,        /* current device is not sm_100             */
+    TRI_ERR_SCRATCH_LIMIT = 10    /* shape needs more than the static scratch */
 } tri_status;
 
 typedef enum tri_format { TRI_TQ1 = 1, TRI_TQ2 = 2 } tri_format;
@@ -193,6 +194,29 @@ TRI_API tri_status tri_gemm_tq2(const uint16_t* X, const uint8_t* qs, const uint
 TRI_API tri_status tri_gemm_tq1(const uint16_t* X, const uint8_t* qs, const uint16_t* d,
                         uint16_t* Y, int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Ternary GEMM without any caller-provided workspace (TQ2, 1 <= M <= 16).
+ * The pages have no counterpart: this is a deployment variant of the
+ * decode-regime kernel for callers that may not allocate device memory (for
+ * example a plugin whose host framework owns all allocations, or code that
+ * runs while a CUDA graph is being captured).
+ *   Same result and argument meaning as tri_gemm_tq2 for these shapes; the
+ *   scratch the kernel needs lives in a static 8 MiB device array inside the
+ *   library, held on every device that loads it until the process exits.
+ *   Returns TRI_ERR_SHAPE for M > 16 and TRI_ERR_SCRATCH_LIMIT when the shape
+ *   needs more scratch than that array holds (tri_gemm_tq2_noalloc_fits
+ *   answers beforehand).  It allocates nothing: the first call on a device
+ *   looks the array up once for that device (and may load the module), so
+ *   make that call before any stream capture.  All calls on a device share
+ *   the array: calls that can run at the same time on that device (other
+ *   streams, other host threads) race, so order them.
+ * ---------------------------------------------------------------------- */
+TRI_API tri_status tri_gemm_tq2_noalloc(const uint16_t* X, const uint8_t* qs, const uint16_t* d,
+                                        uint16_t* Y, int64_t M, int64_t N, int64_t K,
+                                        void* stream);
+/* 1 if tri_gemm_tq2_noalloc accepts this shape on the current device, else 0. */
+TRI_API int tri_gemm_tq2_noalloc_fits(int64_t M, int64_t N, int64_t K);
 
 /* Kernel that tri_gemm would launch for this call under TRI_PATH_AUTO
  * (one of tri_gemm_path), or -1 if the shape is invalid. */

@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(L):
 
 def test_status_strings_and_version(L):
     assert L.tri_version() >= 100
-    for s in range(10):
+    for s in range(11):
         assert L.tri_status_string(s)
     assert L.tri_status_string(12345) == b"unknown status"
 
