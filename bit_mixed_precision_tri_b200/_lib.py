@@ -33,6 +33,7 @@ _f = ctypes.c_float
 SIGNATURES = {
     "tri_status_string": (ctypes.c_char_p, [_i]),
     "tri_version": (_i, []),
+    "tri_last_cuda_error": (ctypes.c_char_p, []),
     "tri_absmean_workspace_bytes": (_sz, [_i64, _i64]),
     "tri_absmean": (_i, [_p, _i64, _i64, _f, _p, _p, _sz, _p]),
     "tri_ternarize": (_i, [_p, _i64, _i64, _f, _p, _p, _p, _sz, _p]),
@@ -84,4 +85,6 @@ def lib() -> ctypes.CDLL:
 
 def check(status: int, what: str) -> None:
     if status != TRI_OK:
+        if status == 6:   # TRI_ERR_CUDA: add the runtime's message
+            what = f"{what} ({lib().tri_last_cuda_error().decode()})"
         raise TriError(status, what)

@@ -1,4 +1,4 @@
-// Compute-regime ternary GEMM (M >= 64) for TQ2 weights on sm_100a.
+// Compute-regime ternary GEMM (M >= 17) for TQ2 weights on sm_100a.
 //
 // Y = X (d * W_hat)^T ("Scaling Laws and Efficient Inference for Ternary
 // Language Models", section "The model", step 3) once the batch is large
@@ -23,8 +23,9 @@
 //
 // The decode emits the pairs (w_j, w_{j+8}) of each 16-weight word, so the
 // activations are consumed in the same within-16 order: a prep kernel writes
-// X once per call in that order (pairs (x_j, x_{j+8}) adjacent), chained to
-// the main kernel with programmatic dependent launch.
+// X once per call in that order (pairs (x_j, x_{j+8}) adjacent) and zeroes
+// the split-K tickets; it is chained to the main kernel with programmatic
+// dependent launch.
 #include <cstdlib>
 
 #include <cudaTypedefs.h>
@@ -59,8 +60,11 @@ struct TcParams {
 
 // ---------------------------------------------------------------- prep kernel
 __global__ void __launch_bounds__(256)
-xperm_kernel(const __half* __restrict__ X, int64_t groups, __half* __restrict__ Xp) {
+xperm_kernel(const __half* __restrict__ X, int64_t groups, __half* __restrict__ Xp,
+             unsigned* __restrict__ tickets, int ntickets) {
   ptx::griddep_launch_dependents();
+  if (blockIdx.x == 0)    // split-K tickets start at zero on every call
+    for (int i = threadIdx.x; i < ntickets; i += blockDim.x) tickets[i] = 0u;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < groups; i += stride) {
     const uint4* src = reinterpret_cast<const uint4*>(X) + 2 * i;
@@ -378,7 +382,8 @@ cudaError_t launch_bn(const Plan& pl, const __half* X, const uint8_t* qs, const 
   const int64_t groups = (int64_t)M * K / 16;
   int64_t gx = ceil_div(groups, 256);
   if (gx > 148 * 8) gx = 148 * 8;
-  xperm_kernel<<<(unsigned)gx, 256, 0, s>>>(X, groups, Xp);
+  xperm_kernel<<<(unsigned)gx, 256, 0, s>>>(X, groups, Xp, reinterpret_cast<unsigned*>(w + pl.off_cnt),
+                                            pl.tiles_n * pl.tiles_m);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 

@@ -32,6 +32,7 @@
 //  * Partial sums of a row tile split across CTAs are combined by the last
 //    CTA to finish (an atomic ticket, no waiting), in CTA order, so results
 //    are deterministic.
+#include <cstdlib>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -43,7 +44,7 @@ namespace tri {
 namespace {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kThreads = kConsumerWarps * 32;   // lane 0 of warp 0 also issues the copies
 constexpr int kBoxRows = 256;                  // TMA box height
 // 16-row mma tiles per consumer warp: four for batches up to 8 (one n8
 // column block), two for batches up to 16 (two column blocks), which keeps
@@ -61,10 +62,11 @@ constexpr int kSmemBudget = 220 * 1024;
 struct Params {
   const uint4* xil;     // [B][MP][32] 16-byte units
   const float* bias;    // [B][MP]
+  const __half* dT;     // [B][Npad] block scales, block-major (prepared per call)
   float* partials;      // [G][2][kRT][MP]
   unsigned* counters;   // [T]
   unsigned* error;      // [1]
-  int M, N, K, B, T, G, stages;
+  int M, N, K, B, T, G, stages, Npad;
   long long U;
 };
 
@@ -76,11 +78,39 @@ __host__ __device__ inline long long cta_of_unit(long long u, long long U, long 
 }
 
 // ---------------------------------------------------------------- prep kernel
+// CTAs [0, B) write the activations of block b in the MMA's pair order (and a
+// bank-conflict-free swizzle) plus the decode bias of each batch row; CTAs
+// [B, B + Npad/64) transpose 64 rows of the scale plane d[N][B] into
+// dT[B][Npad] so that a unit's scales are one contiguous bulk copy.
 template <int MP>
 __global__ void __launch_bounds__(MP * 16)
-xprep_kernel(const __half* __restrict__ X, int M, int K, uint4* __restrict__ xil,
-             float* __restrict__ bias) {
+xprep_kernel(const __half* __restrict__ X, const __half* __restrict__ dsc, int M, int N, int K,
+             int B, int Npad, uint4* __restrict__ xil, float* __restrict__ bias,
+             __half* __restrict__ dT, unsigned* __restrict__ tickets, int T) {
   ptx::griddep_launch_dependents();
+  // the main kernel's per-row-tile tickets start at zero on every call (the
+  // workspace may hold another shape's data); it reads them only after data
+  // that depends on this grid's completion has arrived
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < T; i += blockDim.x) tickets[i] = 0u;
+  if ((int)blockIdx.x >= B) {
+    __shared__ __half tile[64][66];
+    const int r0 = ((int)blockIdx.x - B) * 64;
+    for (int b0 = 0; b0 < B; b0 += 64) {
+      for (int idx = threadIdx.x; idx < 64 * 64; idx += blockDim.x) {
+        const int r = idx >> 6, bb = idx & 63;
+        tile[r][bb] = (r0 + r < N && b0 + bb < B) ? dsc[(size_t)(r0 + r) * B + b0 + bb]
+                                                  : __float2half(0.f);
+      }
+      __syncthreads();
+      for (int idx = threadIdx.x; idx < 64 * 64; idx += blockDim.x) {
+        const int bb = idx >> 6, r = idx & 63;
+        if (b0 + bb < B) dT[(size_t)(b0 + bb) * Npad + r0 + r] = tile[r][bb];
+      }
+      __syncthreads();
+    }
+    return;
+  }
   const int b = blockIdx.x;
   const int m = threadIdx.x >> 4, G = threadIdx.x & 15;
   uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
@@ -138,7 +168,8 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
   uint8_t* wst = smem;                                   // S x kWBytes
   uint8_t* xst = wst + (size_t)S * kWBytes;              // S x kXBytes
   uint8_t* cst = xst + (size_t)S * kXBytes;              // S x kCBytes
-  uint64_t* full = reinterpret_cast<uint64_t*>(cst + (size_t)S * kCBytes);
+  uint8_t* dst_ = cst + (size_t)S * kCBytes;              // S x kRT fp16 scales
+  uint64_t* full = reinterpret_cast<uint64_t*>(dst_ + (size_t)S * kRT * 2);
   uint64_t* empty = full + S;
   volatile int* s_flag = reinterpret_cast<volatile int*>(empty + S);
   volatile int* s_abort = s_flag + 1;
@@ -158,50 +189,46 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
   }
   __syncthreads();
 
-  if (warp == kConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      ptx::prefetch_tensormap(&qmap);
-      const uint64_t pol = ptx::policy_evict_first();
-      const uint32_t tx = kWBytes + kXBytes + MP * 4;
-      const long long n = u1 - u0;
-      const long long pre = n < S ? n : S;
-      uint32_t limit = kWaitLimit;
-      // weights of the first stages do not depend on the prep kernel
-      for (long long i = 0; i < pre; ++i) {
-        const long long u = u0 + i;
-        ptx::mbar_arrive_expect_tx(&full[i], tx);
-        const int bx = (int)(u % B) * 64, ry = (int)(u / B) * kRT;
-        ptx::tma_load_2d(wst + i * kWBytes, &qmap, bx, ry, &full[i], pol);
-        if (Unit<MP>::kBoxes == 2)
-          ptx::tma_load_2d(wst + i * kWBytes + kBoxRows * 64, &qmap, bx, ry + kBoxRows, &full[i], pol);
-      }
-      ptx::griddep_wait();
-      for (long long i = 0; i < pre; ++i) {
-        const int b = (int)((u0 + i) % B);
-        ptx::bulk_load(xst + i * kXBytes, p.xil + (size_t)b * MP * 32, kXBytes, &full[i]);
-        ptx::bulk_load(cst + i * kCBytes, p.bias + (size_t)b * MP, MP * 4, &full[i]);
-      }
-      int s = (int)(pre % S);
-      uint32_t ph = (uint32_t)((pre / S) & 1);
-      int b = (int)((u0 + pre) % B), rt = (int)((u0 + pre) / B);
-      for (long long i = pre; i < n; ++i) {
-        if (!ptx::mbar_wait(&empty[s], ph ^ 1u, limit)) {
-          atomicExch(p.error, 1u);
-          limit = 1;
-        }
-        ptx::mbar_arrive_expect_tx(&full[s], tx);
-        ptx::tma_load_2d(wst + (size_t)s * kWBytes, &qmap, b * 64, rt * kRT, &full[s], pol);
-        if (Unit<MP>::kBoxes == 2)
-          ptx::tma_load_2d(wst + (size_t)s * kWBytes + kBoxRows * 64, &qmap, b * 64, rt * kRT + kBoxRows,
-                           &full[s], pol);
-        ptx::bulk_load(xst + (size_t)s * kXBytes, p.xil + (size_t)b * MP * 32, kXBytes, &full[s]);
-        ptx::bulk_load(cst + (size_t)s * kCBytes, p.bias + (size_t)b * MP, MP * 4, &full[s]);
-        if (++s == S) { s = 0; ph ^= 1u; }
-        if (++b == B) { b = 0; ++rt; }
-      }
+  // ---------------------------------------------------------------- copies
+  // Lane 0 of warp 0 issues every copy: the first S units up front (weights
+  // first: they do not depend on the prep kernel), then one refill per unit,
+  // as soon as all eight warps have released the stage it reuses.
+  const long long n = u1 - u0;
+  const uint32_t tx = kWBytes + kXBytes + MP * 4 + kRT * 2;
+  uint64_t pol = 0;
+  int pb = 0, prt = 0;          // block / row tile of the next unit to load
+  auto issue = [&](int st, int b_, int rt_) {
+    ptx::mbar_arrive_expect_tx(&full[st], tx);
+    ptx::tma_load_2d(wst + (size_t)st * kWBytes, &qmap, b_ * 64, rt_ * kRT, &full[st], pol);
+    if (Unit<MP>::kBoxes == 2)
+      ptx::tma_load_2d(wst + (size_t)st * kWBytes + kBoxRows * 64, &qmap, b_ * 64, rt_ * kRT + kBoxRows,
+                       &full[st], pol);
+    ptx::bulk_load(xst + (size_t)st * kXBytes, p.xil + (size_t)b_ * MP * 32, kXBytes, &full[st]);
+    ptx::bulk_load(cst + (size_t)st * kCBytes, p.bias + (size_t)b_ * MP, MP * 4, &full[st]);
+    ptx::bulk_load(dst_ + (size_t)st * kRT * 2, p.dT + (size_t)b_ * p.Npad + (size_t)rt_ * kRT, kRT * 2,
+                   &full[st]);
+  };
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tensormap(&qmap);
+    pol = ptx::policy_evict_first();
+    const long long pre = n < S ? n : S;
+    for (long long i = 0; i < pre; ++i) {
+      const long long u = u0 + i;
+      ptx::mbar_arrive_expect_tx(&full[i], tx);
+      const int bx = (int)(u % B) * 64, ry = (int)(u / B) * kRT;
+      ptx::tma_load_2d(wst + i * kWBytes, &qmap, bx, ry, &full[i], pol);
+      if (Unit<MP>::kBoxes == 2)
+        ptx::tma_load_2d(wst + i * kWBytes + kBoxRows * 64, &qmap, bx, ry + kBoxRows, &full[i], pol);
     }
-    return;
+    ptx::griddep_wait();        // activations, bias and scales come from the prep kernel
+    for (long long i = 0; i < pre; ++i) {
+      const int b0 = (int)((u0 + i) % B), rt0 = (int)((u0 + i) / B);
+      ptx::bulk_load(xst + i * kXBytes, p.xil + (size_t)b0 * MP * 32, kXBytes, &full[i]);
+      ptx::bulk_load(cst + i * kCBytes, p.bias + (size_t)b0 * MP, MP * 4, &full[i]);
+      ptx::bulk_load(dst_ + i * kRT * 2, p.dT + (size_t)b0 * p.Npad + (size_t)rt0 * kRT, kRT * 2, &full[i]);
+    }
+    pb = (int)((u0 + pre) % B);
+    prt = (int)((u0 + pre) / B);
   }
 
   // -------------------------------------------------------------- consumers
@@ -213,18 +240,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
   int s = 0;
   uint32_t ph = 0;
   int b = (int)(u0 % B), rt = (int)(u0 / B);
-  // scales of the current unit, prefetched one unit ahead
-  float dg[kTiles][2], dn[kTiles][2];
-  auto load_scales = [&](float (&dst)[kTiles][2], int rt_, int b_) {
-#pragma unroll
-    for (int t = 0; t < kTiles; ++t)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int n = rt_ * kRT + warp * kWarpRows + t * 16 + g + 8 * h;
-        dst[t][h] = n < p.N ? __half2float(__ldg(dsc + (size_t)n * B + b_)) : 0.f;
-      }
-  };
-  load_scales(dn, rt, b);
+  float dg[kTiles][2];
   for (long long u = u0; u < u1; ++u) {
     if (u == u0 || b == 0) {
       seg_b0 = b;
@@ -234,13 +250,6 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.f;
-    }
-#pragma unroll
-    for (int t = 0; t < kTiles; ++t) { dg[t][0] = dn[t][0]; dg[t][1] = dn[t][1]; }
-    {
-      int bn = b + 1, rn = rt;
-      if (bn == B) { bn = 0; ++rn; }
-      if (u + 1 < u1) load_scales(dn, rn, bn);
     }
     if (!ptx::mbar_wait(&full[s], ph, limit)) {
       atomicExch(p.error, 2u);
@@ -268,6 +277,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
     }
     // packed words of the warp's rows: rows r and r + 8 of each 16-row tile
     uint32_t wa[kTiles][4], wb[kTiles][4];
+    const __half* ds_s = reinterpret_cast<const __half*>(dst_ + (size_t)s * kRT * 2);
 #pragma unroll
     for (int t = 0; t < kTiles; ++t) {
       const int r = warp * kWarpRows + t * 16 + g;
@@ -275,25 +285,48 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
       const uint4 vb = ptx::lds128(wst_u + (uint32_t)(s * kWBytes + (r + 8) * 64 + 16 * c));
       wa[t][0] = va.x; wa[t][1] = va.y; wa[t][2] = va.z; wa[t][3] = va.w;
       wb[t][0] = vb.x; wb[t][1] = vb.y; wb[t][2] = vb.z; wb[t][3] = vb.w;
+      dg[t][0] = __half2float(ds_s[r]);
+      dg[t][1] = __half2float(ds_s[r + 8]);
     }
-    float C[kTiles][NT][4];
+    // everything this warp needs from the stage is in registers: hand it back
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[s]);
+    if (warp == 0 && lane == 0 && (u - u0) + S < n) {
+      // refill this stage with unit u + S once every warp has released it
+      if (!ptx::mbar_wait(&empty[s], ph, limit)) {
+        atomicExch(p.error, 1u);
+        limit = 1;
+      }
+      issue(s, pb, prt);
+      if (++pb == B) { pb = 0; ++prt; }
+    }
+    __syncwarp();
+    // one accumulator chain per (row tile, 16-group q): 4 x kTiles independent
+    // chains of depth 4, enough to keep the legacy tensor pipe busy (a single
+    // dependent mma.sync chain waits ~140 cycles per step on this part)
+    float C[kTiles][4][NT][4];
 #pragma unroll
     for (int t = 0; t < kTiles; ++t)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        C[t][nt][0] = -cb[nt][0]; C[t][nt][1] = -cb[nt][1];
-        C[t][nt][2] = -cb[nt][0]; C[t][nt][3] = -cb[nt][1];
-      }
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+        for (int nt = 0; nt < NT; ++nt) {
+          C[t][q][nt][0] = q == 0 ? -cb[nt][0] : 0.f;
+          C[t][q][nt][1] = q == 0 ? -cb[nt][1] : 0.f;
+          C[t][q][nt][2] = q == 0 ? -cb[nt][0] : 0.f;
+          C[t][q][nt][3] = q == 0 ? -cb[nt][1] : 0.f;
+        }
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+    for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
           const uint32_t A[4] = {decode_pair(wa[t][q], jj), decode_pair(wb[t][q], jj),
                                  decode_pair(wa[t][q] >> 8, jj), decode_pair(wb[t][q] >> 8, jj)};
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) ptx::mma_16816(C[t][nt], A, bf[nt][q][jj][0], bf[nt][q][jj][1]);
+          for (int nt = 0; nt < NT; ++nt)
+            ptx::mma_16816(C[t][q][nt], A, bf[nt][q][jj][0], bf[nt][q][jj][1]);
         }
       }
     }
@@ -301,13 +334,12 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
     for (int t = 0; t < kTiles; ++t)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        acc[t][nt][0] = fmaf(dg[t][0], C[t][nt][0], acc[t][nt][0]);
-        acc[t][nt][1] = fmaf(dg[t][0], C[t][nt][1], acc[t][nt][1]);
-        acc[t][nt][2] = fmaf(dg[t][1], C[t][nt][2], acc[t][nt][2]);
-        acc[t][nt][3] = fmaf(dg[t][1], C[t][nt][3], acc[t][nt][3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float sum = (C[t][0][nt][e] + C[t][1][nt][e]) + (C[t][2][nt][e] + C[t][3][nt][e]);
+          acc[t][nt][e] = fmaf(dg[t][e >> 1], sum, acc[t][nt][e]);
+        }
       }
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&empty[s]);
     if (++s == S) { s = 0; ph ^= 1u; }
     const int cur_b = b, cur_rt = rt;
     if (++b == B) { b = 0; ++rt; }
@@ -391,7 +423,8 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
 
 // ---------------------------------------------------------------- host side
 struct Layout {
-  size_t off_err, off_cnt, off_xil, off_bias, off_part, total;
+  size_t off_err, off_cnt, off_xil, off_bias, off_dt, off_part, total;
+  int64_t Npad;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -407,7 +440,9 @@ Layout layout_for(int64_t M, int64_t N, int64_t K, int num_sms) {
   L.off_cnt = 256;
   L.off_xil = L.off_cnt + up256((size_t)T * 4);
   L.off_bias = L.off_xil + up256((size_t)B * MP * 512);
-  L.off_part = L.off_bias + up256((size_t)B * MP * 4);
+  L.Npad = T * kRT;
+  L.off_dt = L.off_bias + up256((size_t)B * MP * 4);
+  L.off_part = L.off_dt + up256((size_t)B * L.Npad * 2);
   L.total = L.off_part + up256((size_t)G * 2 * kRT * MP * 4);
   return L;
 }
@@ -425,7 +460,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 int stages_for(int MP) {
-  const int per = (MP == 8 ? Unit<8>::kWBytes : Unit<16>::kWBytes) + MP * 512 + 64;
+  const int rt = MP == 8 ? Unit<8>::kRT : Unit<16>::kRT;
+  const int per = (MP == 8 ? Unit<8>::kWBytes : Unit<16>::kWBytes) + MP * 512 + 64 + rt * 2;
   int s = (kSmemBudget - 2048) / per;
   return s > 12 ? 12 : s;
 }
@@ -446,6 +482,8 @@ cudaError_t launch_mp(const __half* X, const uint8_t* qs, const __half* d, __hal
   p.stages = stages_for(MP);
   p.xil = reinterpret_cast<const uint4*>(w + L.off_xil);
   p.bias = reinterpret_cast<const float*>(w + L.off_bias);
+  p.dT = reinterpret_cast<const __half*>(w + L.off_dt);
+  p.Npad = (int)L.Npad;
   p.partials = reinterpret_cast<float*>(w + L.off_part);
   p.counters = reinterpret_cast<unsigned*>(w + L.off_cnt);
   p.error = reinterpret_cast<unsigned*>(w + L.off_err);
@@ -462,12 +500,13 @@ cudaError_t launch_mp(const __half* X, const uint8_t* qs, const __half* d, __hal
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
-  xprep_kernel<MP><<<p.B, MP * 16, 0, s>>>(X, M, K, reinterpret_cast<uint4*>(w + L.off_xil),
-                                          reinterpret_cast<float*>(w + L.off_bias));
+  xprep_kernel<MP><<<p.B + p.Npad / 64, MP * 16, 0, s>>>(
+      X, d, M, N, K, p.B, p.Npad, reinterpret_cast<uint4*>(w + L.off_xil),
+      reinterpret_cast<float*>(w + L.off_bias), reinterpret_cast<__half*>(w + L.off_dt), p.counters, p.T);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  const size_t smem = (size_t)p.stages * (kWBytes + MP * 512 + 64) + 2 * p.stages * 8 + 16 + 1024;
+  const size_t smem = (size_t)p.stages * (kWBytes + MP * 512 + 64 + kRT * 2) + 2 * p.stages * 8 + 16 + 1024;
   e = cudaFuncSetAttribute(gemv_mma_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -485,17 +524,26 @@ cudaError_t launch_mp(const __half* X, const uint8_t* qs, const __half* d, __hal
 
 }  // namespace
 
+// The decode-regime path runs the mma.sync kernel above; the tcgen05 kernel
+// (gemv_tc.cu) is selectable for comparison (TRI_DECODE_KERNEL=tc).
+bool use_legacy_decode() {
+  const char* e = std::getenv("TRI_DECODE_KERNEL");
+  return !(e && e[0] == 't');
+}
+
 bool gemv_mma_supported(int fmt, int64_t M, int64_t N, int64_t K) {
   return fmt == TRI_TQ2 && M >= 1 && M <= 16 && N >= 1 && K >= kBlock && K % kBlock == 0;
 }
 
 size_t gemv_mma_ws_bytes(int, int64_t M, int64_t N, int64_t K, int num_sms) {
-  return layout_for(M, N, K, num_sms).total;
+  const size_t a = layout_for(M, N, K, num_sms).total, b = gemv_tc_ws_bytes(N, K, num_sms);
+  return a > b ? a : b;
 }
 
 cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const __half* d, __half* Y,
                             int M, int N, int K, void* ws, int num_sms, cudaStream_t s) {
   if (!gemv_mma_supported(fmt, M, N, K)) return cudaErrorNotSupported;
+  if (!use_legacy_decode()) return launch_gemv_tc(X, qs, d, Y, M, N, K, ws, num_sms, s);
   if (M <= 8) return launch_mp<8>(X, qs, d, Y, M, N, K, ws, num_sms, s);
   return launch_mp<16>(X, qs, d, Y, M, N, K, ws, num_sms, s);
 }
@@ -532,7 +580,7 @@ std::once_flag g_scratch_once[kMaxDev];
 size_t gemv_noalloc_scratch_limit() { return kNoAllocScratchBytes; }
 
 size_t gemv_noalloc_scratch_need(int64_t M, int64_t N, int64_t K, int num_sms) {
-  return layout_for(M, N, K, num_sms).total;
+  return gemv_mma_ws_bytes(TRI_TQ2, M, N, K, num_sms);
 }
 
 cudaError_t launch_gemv_mma_noalloc(const __half* X, const uint8_t* qs, const __half* d, __half* Y,
@@ -547,11 +595,11 @@ cudaError_t launch_gemv_mma_noalloc(const __half* X, const uint8_t* qs, const __
     g_scratch_addr[dev] = ptr;
   });
   if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
-  const Layout L = layout_for(M, N, K, num_sms);
-  if (L.total > kNoAllocScratchBytes) return cudaErrorInvalidValue;
+  if (gemv_noalloc_scratch_need(M, N, K, num_sms) > kNoAllocScratchBytes) return cudaErrorInvalidValue;
   uint8_t* ws = static_cast<uint8_t*>(g_scratch_addr[dev]);
-  // the tickets must start at zero; the array keeps whatever the last call left
-  e = cudaMemsetAsync(ws + L.off_cnt, 0, L.off_xil - L.off_cnt, s);
+  // the tickets (one per 128-row tile, after a 256-byte header in both decode
+  // kernels' layouts) must start at zero; the array keeps the last call's bytes
+  e = cudaMemsetAsync(ws + 256, 0, up256((size_t)ceil_div(N, 128) * 4), s);
   if (e != cudaSuccess) return e;
   return launch_gemv_mma(TRI_TQ2, X, qs, d, Y, M, N, K, ws, num_sms, s);
 }

@@ -40,8 +40,11 @@ tri_status device_info(DevInfo* out) {
   return TRI_OK;
 }
 
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
 tri_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return TRI_OK;
+  g_last_cuda = e;
   cudaGetLastError();
   return TRI_ERR_CUDA;
 }
@@ -53,11 +56,34 @@ tri_status check_nk(int64_t N, int64_t K) {
   return TRI_OK;
 }
 
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// The tensor-core kernels consume TQ2 planes; TQ1 weights reach them through
+// a transcode into the head of the workspace (N*K/4 bytes).
+bool path_supported(int fmt, int path, int64_t M, int64_t N, int64_t K) {
+  (void)fmt;
+  switch (path) {
+    case TRI_PATH_SIMT: return true;
+    case TRI_PATH_MMA: return tri::gemv_mma_supported(TRI_TQ2, M, N, K);
+    case TRI_PATH_TCGEN05: return tri::gemm_tc_supported(TRI_TQ2, M, N, K);
+    default: return false;
+  }
+}
+
+size_t transcode_bytes(int fmt, int path, int64_t N, int64_t K) {
+  return (fmt == TRI_TQ1 && path != TRI_PATH_SIMT) ? up256((size_t)N * (size_t)K / 4) : 0;
+}
+
+size_t path_ws_bytes(int fmt, int path, int64_t M, int64_t N, int64_t K, int sms) {
+  size_t inner = 0;
+  if (path == TRI_PATH_MMA) inner = tri::gemv_mma_ws_bytes(TRI_TQ2, M, N, K, sms);
+  if (path == TRI_PATH_TCGEN05) inner = tri::gemm_tc_ws_bytes(TRI_TQ2, M, N, K, sms);
+  return transcode_bytes(fmt, path, N, K) + inner;
+}
+
 int auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
-  if (M <= 16 && tri::gemv_mma_supported(fmt, M, N, K)) return TRI_PATH_MMA;
-  if (M >= 64 && tri::gemm_tc_supported(fmt, M, N, K)) return TRI_PATH_TCGEN05;
-  if (tri::gemm_tc_supported(fmt, M, N, K) && M > 16) return TRI_PATH_TCGEN05;
-  if (tri::gemv_mma_supported(fmt, M, N, K)) return TRI_PATH_MMA;
+  if (M <= 16 && path_supported(fmt, TRI_PATH_MMA, M, N, K)) return TRI_PATH_MMA;
+  if (M > 16 && path_supported(fmt, TRI_PATH_TCGEN05, M, N, K)) return TRI_PATH_TCGEN05;
   return TRI_PATH_SIMT;
 }
 
@@ -83,6 +109,8 @@ const char* tri_status_string(int status) {
 }
 
 int tri_version(void) { return 100; }
+
+const char* tri_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
 
 size_t tri_absmean_workspace_bytes(int64_t, int64_t) { return tri::absmean_ws_bytes(); }
 
@@ -165,9 +193,12 @@ size_t tri_gemm_workspace_bytes(int format, int64_t M, int64_t N, int64_t K) {
   DevInfo di;
   int sms = 148;
   if (device_info(&di) == TRI_OK) sms = di.sms;
-  size_t a = tri::gemv_mma_supported(format, M, N, K) ? tri::gemv_mma_ws_bytes(format, M, N, K, sms) : 0;
-  size_t b = tri::gemm_tc_supported(format, M, N, K) ? tri::gemm_tc_ws_bytes(format, M, N, K, sms) : 0;
-  size_t r = a > b ? a : b;
+  size_t r = 0;
+  for (int path = TRI_PATH_SIMT; path <= TRI_PATH_TCGEN05; ++path)
+    if (path_supported(format, path, M, N, K)) {
+      const size_t b = path_ws_bytes(format, path, M, N, K, sms);
+      if (b > r) r = b;
+    }
   return r < 256 ? 256 : r;
 }
 
@@ -185,29 +216,32 @@ tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs, 
   DevInfo di;
   if ((st = device_info(&di)) != TRI_OK) return st;
   if (path == TRI_PATH_AUTO) path = auto_path(format, M, N, K);
+  if (!path_supported(format, path, M, N, K)) return TRI_ERR_NOT_IMPLEMENTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __half* Xh = reinterpret_cast<const __half*>(X);
   const __half* dh = reinterpret_cast<const __half*>(d);
   __half* Yh = reinterpret_cast<__half*>(Y);
+  if (path == TRI_PATH_SIMT)
+    return from_cuda(tri::launch_gemm_simt(format, Xh, qs, dh, Yh, (int)M, (int)N, (int)K, s));
+  const size_t need = path_ws_bytes(format, path, M, N, K, di.sms);
+  if (need && (!workspace || workspace_bytes < need)) return TRI_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
+  const uint8_t* q2 = qs;
+  uint8_t* inner = static_cast<uint8_t*>(workspace);
+  if (format == TRI_TQ1) {
+    uint8_t* t = static_cast<uint8_t*>(workspace);
+    const cudaError_t e = tri::launch_transcode_tq1_tq2(qs, N, K, t, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    q2 = t;
+    inner = t + transcode_bytes(format, path, N, K);
+  }
   switch (path) {
-    case TRI_PATH_SIMT:
-      return from_cuda(tri::launch_gemm_simt(format, Xh, qs, dh, Yh, (int)M, (int)N, (int)K, s));
-    case TRI_PATH_MMA: {
-      if (!tri::gemv_mma_supported(format, M, N, K)) return TRI_ERR_NOT_IMPLEMENTED;
-      const size_t need = tri::gemv_mma_ws_bytes(format, M, N, K, di.sms);
-      if (need && (!workspace || workspace_bytes < need)) return TRI_ERR_WORKSPACE;
-      if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
-      return from_cuda(tri::launch_gemv_mma(format, Xh, qs, dh, Yh, (int)M, (int)N, (int)K,
-                                            workspace, di.sms, s));
-    }
-    case TRI_PATH_TCGEN05: {
-      if (!tri::gemm_tc_supported(format, M, N, K)) return TRI_ERR_NOT_IMPLEMENTED;
-      const size_t need = tri::gemm_tc_ws_bytes(format, M, N, K, di.sms);
-      if (need && (!workspace || workspace_bytes < need)) return TRI_ERR_WORKSPACE;
-      if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
-      return from_cuda(tri::launch_gemm_tc(format, Xh, qs, dh, Yh, (int)M, (int)N, (int)K,
-                                           workspace, di.sms, s));
-    }
+    case TRI_PATH_MMA:
+      return from_cuda(tri::launch_gemv_mma(TRI_TQ2, Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner,
+                                            di.sms, s));
+    case TRI_PATH_TCGEN05:
+      return from_cuda(tri::launch_gemm_tc(TRI_TQ2, Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner,
+                                           di.sms, s));
     default:
       return TRI_ERR_INVALID_ARG;
   }

@@ -35,6 +35,10 @@ cudaError_t launch_unpack_tq2(const uint8_t* qs, int64_t N, int64_t K, int8_t* t
 cudaError_t launch_unpack_tq1(const uint8_t* qs, int64_t N, int64_t K, int8_t* trits,
                               int32_t* invalid, cudaStream_t s);
 
+// TQ1 plane -> TQ2 plane (N*K/4 bytes, 16-B aligned), for the tensor-core paths
+cudaError_t launch_transcode_tq1_tq2(const uint8_t* qs1, int64_t N, int64_t K, uint8_t* qs2,
+                                     cudaStream_t s);
+
 cudaError_t launch_gemm_simt(int fmt, const __half* X, const uint8_t* qs, const __half* d,
                              __half* Y, int M, int N, int K, cudaStream_t s);
 
@@ -44,6 +48,11 @@ size_t gemv_mma_ws_bytes(int fmt, int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const __half* d,
                             __half* Y, int M, int N, int K, void* ws, int num_sms,
                             cudaStream_t s);
+
+// decode-regime kernel on tcgen05 with decoded weights in tensor memory (TQ2, M <= 16)
+size_t gemv_tc_ws_bytes(int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv_tc(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M, int N,
+                           int K, void* ws, int num_sms, cudaStream_t s);
 
 // decode-regime path with library-owned static scratch (no allocation)
 size_t gemv_noalloc_scratch_limit();

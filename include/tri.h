@@ -91,6 +91,10 @@ TRI_API const char* tri_status_string(int status);
 /* Library ABI version (major*100 + minor). */
 TRI_API int tri_version(void);
 
+/* The CUDA runtime's message for the last error behind a TRI_ERR_CUDA
+ * returned on the calling host thread (static string, never NULL). */
+TRI_API const char* tri_last_cuda_error(void);
+
 /* ------------------------------------------------------------------------
  * Absmean scale ("The model", step 1; Spectra "Architecture": one scale per
  * matrix, the mean absolute value of the latent weights).
@@ -176,9 +180,9 @@ TRI_API tri_status tri_unpack(int format, const uint8_t* qs, int64_t N, int64_t 
  *   Y         device fp16[M][N], 16-byte aligned, written.
  *   M >= 1, N >= 1, K >= 256 with K % 256 == 0; M, N, K < 2^31.
  *   workspace device scratch of at least tri_gemm_workspace_bytes(format, M,
- *             N, K) bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE
- *             (the kernels leave it zeroed for the next call).  Calls that
- *             share one workspace must be ordered (same stream, or events).
+ *             N, K) bytes, 256-byte aligned; its contents on entry do not
+ *             matter (each call initialises what it uses).  Calls that share
+ *             one workspace must be ordered (same stream, or events).
  *   path      TRI_PATH_AUTO chooses TRI_PATH_MMA for M <= 16 and
  *             TRI_PATH_TCGEN05 for M >= 64 (TQ2; TQ1 for M >= 64 too), else
  *             the best available; an explicit path that cannot serve the
