@@ -51,7 +51,7 @@ WORKLOADS = {
 }
 # path -> launches of this library's kernels per GEMM call (prep + main for the
 # tensor-core paths; TQ1 adds its transcode)
-KERNELS_PER_CALL = {1: 1, 2: 2, 3: 2}
+KERNELS_PER_CALL = {1: 1, 2: 2, 3: 2, 4: 2}
 
 
 def workload_from_args(name, M=None, fmt=None):

@@ -5,6 +5,6 @@ The torch-facing functions live in ``api``; they load ``libtri_b200.so``
 (built in-tree by ``build.py``) on first use.
 """
 from .api import (  # noqa: F401
-    PATH_AUTO, PATH_MMA, PATH_SIMT, PATH_TCGEN05, TernaryLinear, TriError, Workspace, absmean,
+    PATH_AUTO, PATH_I8, PATH_MMA, PATH_SIMT, PATH_TCGEN05, TernaryLinear, TriError, Workspace, absmean,
     auto_path, gemm, gemm_workspace_bytes, pack, packed_row_bytes, ternarize, unpack,
 )

@@ -17,7 +17,7 @@ HEADER = os.path.join(ROOT, "include", "tri.h")
 
 TRI_OK = 0
 TRI_TQ1, TRI_TQ2 = 1, 2
-PATH_AUTO, PATH_SIMT, PATH_MMA, PATH_TCGEN05 = 0, 1, 2, 3
+PATH_AUTO, PATH_SIMT, PATH_MMA, PATH_TCGEN05, PATH_I8 = 0, 1, 2, 3, 4
 STATUS_NAMES = {
     0: "TRI_OK", 1: "TRI_ERR_INVALID_ARG", 2: "TRI_ERR_SHAPE", 3: "TRI_ERR_ALIGNMENT",
     4: "TRI_ERR_NONFINITE", 5: "TRI_ERR_INVALID_CODE", 6: "TRI_ERR_CUDA",

@@ -9,7 +9,7 @@ from __future__ import annotations
 import torch
 
 from . import _lib
-from ._lib import PATH_AUTO, PATH_MMA, PATH_SIMT, PATH_TCGEN05, TRI_TQ1, TRI_TQ2, TriError  # noqa: F401
+from ._lib import PATH_AUTO, PATH_I8, PATH_MMA, PATH_SIMT, PATH_TCGEN05, TRI_TQ1, TRI_TQ2, TriError  # noqa: F401
 
 FORMATS = {"tq2": TRI_TQ2, "tq1": TRI_TQ1}
 

@@ -66,6 +66,7 @@ bool path_supported(int fmt, int path, int64_t M, int64_t N, int64_t K) {
     case TRI_PATH_SIMT: return true;
     case TRI_PATH_MMA: return tri::gemv_mma_supported(TRI_TQ2, M, N, K);
     case TRI_PATH_TCGEN05: return tri::gemm_tc_supported(TRI_TQ2, M, N, K);
+    case TRI_PATH_I8: return tri::gemv_i8_supported(M, N, K);
     default: return false;
   }
 }
@@ -78,10 +79,12 @@ size_t path_ws_bytes(int fmt, int path, int64_t M, int64_t N, int64_t K, int sms
   size_t inner = 0;
   if (path == TRI_PATH_MMA) inner = tri::gemv_mma_ws_bytes(TRI_TQ2, M, N, K, sms);
   if (path == TRI_PATH_TCGEN05) inner = tri::gemm_tc_ws_bytes(TRI_TQ2, M, N, K, sms);
+  if (path == TRI_PATH_I8) inner = tri::gemv_i8_ws_bytes(M, N, K, sms);
   return transcode_bytes(fmt, path, N, K) + inner;
 }
 
 int auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
+  if (M <= 2 && path_supported(fmt, TRI_PATH_I8, M, N, K)) return TRI_PATH_I8;
   if (M <= 16 && path_supported(fmt, TRI_PATH_MMA, M, N, K)) return TRI_PATH_MMA;
   if (M > 16 && path_supported(fmt, TRI_PATH_TCGEN05, M, N, K)) return TRI_PATH_TCGEN05;
   return TRI_PATH_SIMT;
@@ -194,7 +197,7 @@ size_t tri_gemm_workspace_bytes(int format, int64_t M, int64_t N, int64_t K) {
   int sms = 148;
   if (device_info(&di) == TRI_OK) sms = di.sms;
   size_t r = 0;
-  for (int path = TRI_PATH_SIMT; path <= TRI_PATH_TCGEN05; ++path)
+  for (int path = TRI_PATH_SIMT; path <= TRI_PATH_I8; ++path)
     if (path_supported(format, path, M, N, K)) {
       const size_t b = path_ws_bytes(format, path, M, N, K, sms);
       if (b > r) r = b;
@@ -206,7 +209,7 @@ tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs, 
                     uint16_t* Y, int64_t M, int64_t N, int64_t K, void* workspace,
                     size_t workspace_bytes, void* stream) {
   if (format != TRI_TQ2 && format != TRI_TQ1) return TRI_ERR_INVALID_ARG;
-  if (path < TRI_PATH_AUTO || path > TRI_PATH_TCGEN05) return TRI_ERR_INVALID_ARG;
+  if (path < TRI_PATH_AUTO || path > TRI_PATH_I8) return TRI_ERR_INVALID_ARG;
   if (!X || !qs || !d || !Y) return TRI_ERR_INVALID_ARG;
   if (M < 1 || M > kMaxDim) return TRI_ERR_SHAPE;
   tri_status st = check_nk(N, K);
@@ -239,6 +242,8 @@ tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs, 
     case TRI_PATH_MMA:
       return from_cuda(tri::launch_gemv_mma(TRI_TQ2, Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner,
                                             di.sms, s));
+    case TRI_PATH_I8:
+      return from_cuda(tri::launch_gemv_i8(Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner, di.sms, s));
     case TRI_PATH_TCGEN05:
       return from_cuda(tri::launch_gemm_tc(TRI_TQ2, Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner,
                                            di.sms, s));

@@ -84,5 +84,5 @@ def test_auto_path_and_workspace_query(L):
     for fmt in (1, 2):
         for M in (1, 16, 64, 256):
             p = L.tri_gemm_auto_path(fmt, M, 4096, 4096)
-            assert p in (1, 2, 3)
+            assert p in (1, 2, 3, 4)
             assert L.tri_gemm_workspace_bytes(fmt, M, 4096, 4096) >= 256

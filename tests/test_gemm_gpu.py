@@ -12,7 +12,8 @@ from oracle import tri_oracle as O
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
-PATHS = {"simt": tri.PATH_SIMT, "mma": tri.PATH_MMA, "tcgen05": tri.PATH_TCGEN05}
+PATHS = {"simt": tri.PATH_SIMT, "i8": tri.PATH_I8, "mma": tri.PATH_MMA,
+         "tcgen05": tri.PATH_TCGEN05}
 
 
 def _supported(path, fmt, M, N, K):
@@ -151,4 +152,45 @@ def test_gemm_repeat_deterministic():
             N, K, "tq2")
     Y1 = tri.gemm(*args)
     Y2 = tri.gemm(*args)
+    assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+@pytest.mark.parametrize("M,N,K", [(1, 65536, 1024), (2, 1000, 11008), (1, 129, 256), (2, 3, 512)])
+def test_i8_path_shapes(fmt, M, N, K):
+    """The integer path at shapes that exercise its work split: more units per
+    CTA than block pairs per row (slot wrap), an odd number of blocks per row
+    (a half-empty last pair), ragged row tiles and a grid smaller than the SMs."""
+    X, trits, qs, d = _case(M, N, K, 300 + M + N % 97, fmt, per_block=True, p_zero=0.31)
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, fmt, path=tri.PATH_I8)
+    _check(Y, X, trits, d)
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_i8_path_activation_extremes(M):
+    """Fixed-point activations: a block holding one value near the fp16 maximum
+    among tiny ones (the quantisation step is set by the largest |x| of the
+    block), an all-zero block, subnormal values and signed extremes."""
+    N, K = 384, 2048
+    X, trits, qs, d = _case(M, N, K, 41, "tq2", per_block=True, p_zero=0.5)
+    X = X.copy()
+    X[:, 0] = 60000.0
+    X[:, 1:256] = (np.random.default_rng(3).standard_normal((M, 255)) * 1e-3).astype(np.float16)
+    X[:, 256:512] = 0.0
+    X[:, 512:768] = np.float16(6e-8)
+    X[:, 768] = -65504.0
+    X[:, 769] = 65504.0
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, "tq2", path=tri.PATH_I8)
+    _check(Y, X, trits, d)
+
+
+def test_i8_path_deterministic():
+    M, N, K = 1, 8192, 28672 // 4
+    X, trits, qs, d = _case(M, N, K, 9, "tq2")
+    args = (torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV),
+            N, K, "tq2")
+    Y1 = tri.gemm(*args, path=tri.PATH_I8)
+    Y2 = tri.gemm(*args, path=tri.PATH_I8)
     assert torch.equal(Y1, Y2)
