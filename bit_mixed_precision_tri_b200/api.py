@@ -110,8 +110,8 @@ def auto_path(fmt, M: int, N: int, K: int) -> int:
 
 
 class Workspace:
-    """Zero-filled device scratch for tri_gemm, grown on demand (kept zeroed
-    by the kernels between calls)."""
+    """Device scratch for tri_gemm, grown on demand.  Its contents between
+    calls do not matter; calls that share one must be ordered (one stream)."""
 
     def __init__(self, device=None):
         self.device = torch.device(device or "cuda")

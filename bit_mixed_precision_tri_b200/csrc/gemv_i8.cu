@@ -34,15 +34,22 @@
 //    keeps four units of 16-byte cp.async copies in flight.  A row tile split
 //    between CTAs is summed, in CTA order (deterministic), by the CTA that
 //    holds its first unit; the others leave partial sums stamped with the
-//    call's generation number (one 64-bit store each: no fence, no atomic),
-//    so bytes left in the workspace by earlier calls never pass for them and
-//    the workspace needs no clearing.
-#include <atomic>
+//    call's epoch (one 64-bit store each: no fence, no atomic).  The epoch is
+//    a counter on the device, one per workspace in a small library-owned
+//    pool, advanced by the last CTA of each call: bytes left in the
+//    workspace by earlier calls never pass for this call's sums, the
+//    workspace needs no clearing, and a captured graph replays correctly.
+#include <mutex>
 
 #include "sm100_ptx.cuh"
 #include "tri_internal.cuh"
 
 namespace tri {
+
+constexpr int kEpochSlots = 64;        // workspaces with an epoch slot per device
+// [slot][0]: epoch of the next call, [slot][1]: CTAs of the current call done
+static __device__ unsigned g_i8_epochs[kEpochSlots][2];
+
 namespace {
 
 constexpr int kWarps = 8;
@@ -52,8 +59,9 @@ constexpr float kQMax = 8.0e6f;        // |x^| bound: three balanced base-256 di
 
 struct Params {
   const __half* X;       // [M][K]
-  unsigned long long* partials;  // [G][kRT][M]: generation << 32 | fp32 bits
-  unsigned long long gen;        // this call's generation (32 bits, never 0)
+  unsigned long long* partials;  // [G][kRT][M]: stamp << 32 | fp32 bits
+  unsigned* epoch;       // this workspace's [epoch, done] pair in the pool
+  unsigned slot;         // its index (part of every stamp)
   unsigned* error;       // set when a wait for a partial sum gives up (never expected)
   int N, K, B, P, T, G;
   long long U;
@@ -204,6 +212,9 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
   // the grid, so none of its slots may go to a later grid first.
   issue(0, true);                                     // group 0: weight stage 0
   ptx::griddep_wait();
+  // this call's stamp: epoch and slot (the previous grid's epoch update is visible now)
+  const unsigned long long stamp =
+      (unsigned long long)((*reinterpret_cast<volatile unsigned*>(p.epoch) + 1u) * (unsigned)kEpochSlots + p.slot);
   const int n_pairs = n_units < P ? n_units : P;
   {
     // zero slots, read by the lanes without a B column
@@ -351,11 +362,11 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
         for (int m = 0; m < M; ++m) {
           const unsigned long long* a = src + (r_local + 8 * h) * M + m;
           unsigned long long v = ld_relaxed_u64(a);
-          for (int spin = 0; (v >> 32) != p.gen && spin < kSpinLimit; ++spin) {
+          for (int spin = 0; (v >> 32) != stamp && spin < kSpinLimit; ++spin) {
             __nanosleep(64);
             v = ld_relaxed_u64(a);
           }
-          if ((v >> 32) != p.gen) atomicOr(p.error, 1u);
+          if ((v >> 32) != stamp) atomicOr(p.error, 1u);
           sum[h][m] += __uint_as_float((unsigned)v);
         }
     }
@@ -464,7 +475,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int m = 0; m < M; ++m)
-              __stcg(mine + (r_local + 8 * h) * M + m, (p.gen << 32) | __float_as_uint(acc[h][m]));
+              __stcg(mine + (r_local + 8 * h) * M + m, (stamp << 32) | __float_as_uint(acc[h][m]));
         }
       }
 #pragma unroll
@@ -475,7 +486,12 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
     }
   }
   cp_async_wait<0>();
-
+  // the last CTA to finish advances the epoch for the next call on this workspace
+  __syncthreads();
+  if (threadIdx.x == 0 && atomicAdd(&p.epoch[1], 1u) == (unsigned)(p.G - 1)) {
+    p.epoch[1] = 0u;
+    p.epoch[0] = p.epoch[0] + 1u;
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -516,8 +532,46 @@ Layout layout_for(int64_t M, int64_t N, int64_t K, int num_sms) {
   return M == 1 ? layout_m<1>(N, K, num_sms) : layout_m<2>(N, K, num_sms);
 }
 
-// generation numbers of the calls (32 bits, starting at 1; one per launch)
-std::atomic<unsigned long long> g_generation{0};
+// ---- epoch slots: one per (device, workspace); the least recently used is reused
+struct SlotTable {
+  std::mutex mu;
+  const void* ws[kEpochSlots] = {};
+  unsigned long long used[kEpochSlots] = {};
+  unsigned long long clock = 0;
+  unsigned* base = nullptr;
+};
+constexpr int kMaxDev = 64;
+SlotTable g_slots[kMaxDev];
+
+cudaError_t epoch_slot(const void* ws, unsigned** out, unsigned* slot_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  SlotTable& t = g_slots[dev];
+  std::lock_guard<std::mutex> lock(t.mu);
+  if (!t.base) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_i8_epochs);
+    if (e != cudaSuccess) return e;
+    t.base = static_cast<unsigned*>(ptr);
+  }
+  int slot = -1, lru = 0;
+  for (int i = 0; i < kEpochSlots; ++i) {
+    if (t.ws[i] == ws) { slot = i; break; }
+    if (t.used[i] < t.used[lru]) lru = i;
+  }
+  if (slot < 0) {
+    // a reused slot keeps counting: stamps carry the slot index, so sums that
+    // an earlier workspace left under another slot can never match
+    slot = lru;
+    t.ws[slot] = ws;
+  }
+  t.used[slot] = ++t.clock;
+  *out = t.base + 2 * slot;
+  *slot_out = (unsigned)slot;
+  return cudaSuccess;
+}
 
 template <int M>
 cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int N, int K,
@@ -527,9 +581,8 @@ cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half
   Params p;
   p.X = X;
   p.partials = reinterpret_cast<unsigned long long*>(w + L.off_part);
-  p.gen = (g_generation.fetch_add(1) + 1) & 0xFFFFFFFFull;
-  if (p.gen == 0) p.gen = g_generation.fetch_add(1) + 1;   // 0 is skipped on wrap-around
-  p.gen &= 0xFFFFFFFFull;
+  cudaError_t e0 = epoch_slot(ws, &p.epoch, &p.slot);
+  if (e0 != cudaSuccess) return e0;
   p.error = reinterpret_cast<unsigned*>(w + L.off_err);
   p.N = N; p.K = K; p.B = K / kBlock; p.P = L.P; p.T = L.T; p.G = L.G; p.U = L.U;
   p.k4 = 4; p.k16 = 16; p.k64 = 64;

@@ -194,3 +194,42 @@ def test_i8_path_deterministic():
     Y1 = tri.gemm(*args, path=tri.PATH_I8)
     Y2 = tri.gemm(*args, path=tri.PATH_I8)
     assert torch.equal(Y1, Y2)
+
+
+def test_i8_path_graph_replay_new_inputs():
+    """A captured call replayed with new activations in the same buffers: the
+    split-tile partial sums of one replay must never stand in for the next's."""
+    M, N, K = 1, 4096, 7168
+    X, trits, qs, d = _case(M, N, K, 61, "tq2")
+    Xd = torch.from_numpy(X).to(DEV)
+    qd, dd = torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV)
+    Y = torch.empty(M, N, dtype=torch.float16, device=DEV)
+    ws = tri.Workspace(DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        tri.gemm(Xd, qd, dd, N, K, "tq2", out=Y, workspace=ws, stream=s, path=tri.PATH_I8)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        tri.gemm(Xd, qd, dd, N, K, "tq2", out=Y, workspace=ws, stream=s, path=tri.PATH_I8)
+    for seed in (7, 8, 9):
+        Xn = inputs.activations(M, K, seed).numpy()
+        Xd.copy_(torch.from_numpy(Xn).to(DEV))
+        g.replay()
+        torch.cuda.synchronize()
+        _check(Y, Xn, trits, d)
+
+
+def test_i8_path_workspace_shared_with_other_paths():
+    """The same workspace alternates between the integer path and the others
+    (which leave their own bytes in it): results stay correct."""
+    N, K = 2048, 7168
+    X1, trits, qs, d = _case(1, N, K, 62, "tq2", per_block=True, p_zero=0.4)
+    X8 = inputs.activations(8, K, 63).numpy()
+    qd, dd = torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV)
+    ws = tri.Workspace(DEV)
+    for rep in range(3):
+        Y1 = tri.gemm(torch.from_numpy(X1).to(DEV), qd, dd, N, K, "tq2", workspace=ws, path=tri.PATH_I8)
+        _check(Y1, X1, trits, d)
+        Y8 = tri.gemm(torch.from_numpy(X8).to(DEV), qd, dd, N, K, "tq2", workspace=ws, path=tri.PATH_MMA)
+        _check(Y8, X8, trits, d)
