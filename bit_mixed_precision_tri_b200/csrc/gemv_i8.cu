@@ -207,9 +207,12 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
     if (commit) cp_async_commit();                    // one group per stage (empty at the end)
   };
   // The weights do not depend on X: the first stage is copied before waiting
-  // for the grid that produced X (programmatic dependent launch).  This grid
-  // never triggers its dependents early: a reducer waits for other CTAs of
-  // the grid, so none of its slots may go to a later grid first.
+  // for the grid that produced X (programmatic dependent launch).  Every CTA
+  // lets the next grid launch as soon as it runs: that grid can only start
+  // once all CTAs of this one have done so, i.e. are resident, so its CTAs
+  // never take a slot that a CTA of this grid (which a reducer may wait for)
+  // still needs.
+  ptx::griddep_launch_dependents();
   issue(0, true);                                     // group 0: weight stage 0
   ptx::griddep_wait();
   // this call's stamp: epoch and slot (the previous grid's epoch update is visible now)
@@ -573,6 +576,28 @@ cudaError_t epoch_slot(const void* ws, unsigned** out, unsigned* slot_out) {
   return cudaSuccess;
 }
 
+// the kernel's dynamic shared memory limit, raised once per device to the
+// largest size any supported shape uses
+template <int M>
+size_t smem_limit() {
+  return (size_t)Cfg<M>::kRing + (size_t)Cfg<M>::kMaxPairs * Cfg<M>::kPairBytes;
+}
+
+template <int M>
+cudaError_t smem_attribute() {
+  static std::once_flag once[kMaxDev];
+  static cudaError_t err[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  std::call_once(once[dev], [dev]() {
+    err[dev] = cudaFuncSetAttribute(gemv_i8_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem_limit<M>());
+  });
+  return err[dev];
+}
+
 template <int M>
 cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int N, int K,
                      void* ws, int num_sms, cudaStream_t s) {
@@ -586,7 +611,7 @@ cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half
   p.error = reinterpret_cast<unsigned*>(w + L.off_err);
   p.N = N; p.K = K; p.B = K / kBlock; p.P = L.P; p.T = L.T; p.G = L.G; p.U = L.U;
   p.k4 = 4; p.k16 = 16; p.k64 = 64;
-  cudaError_t e = cudaFuncSetAttribute(gemv_i8_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.smem);
+  cudaError_t e = smem_attribute<M>();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)L.G);
