@@ -159,10 +159,17 @@ def prepare_layers(w, device, copies):
     from bit_mixed_precision_tri_b200 import inputs
     layers = []
     for (N, K), seed in zip(w["layers"], w["seeds"]):
-        W = inputs.latent_weights(N, K, seed).to(device)
-        trits, g = tri.ternarize(W, 1e-6)
-        qs, d = tri.pack(trits, g, w["fmt"])
-        del W, trits
+        if w.get("p_zero") is None:
+            W = inputs.latent_weights(N, K, seed).to(device)
+            trits, g = tri.ternarize(W, 1e-6)
+            qs, d = tri.pack(trits, g, w["fmt"])
+            del W
+        else:   # format stress: i.i.d. trits, one scale per 256-block
+            trits = inputs.random_trits(N, K, w["p_zero"], seed).to(device)
+            g = inputs.block_scales(N, K, seed + 1).to(device)
+            qs, d = tri.pack(trits, g, w["fmt"])
+            g = g.max()
+        del trits
         reps = [(qs, d)] + [(qs.clone(), d.clone()) for _ in range(copies - 1)]
         X = inputs.activations(w["M"], K, 6 + w["M"] + seed).to(device)
         Y = torch.empty(w["M"], N, dtype=torch.float16, device=device)
@@ -171,9 +178,10 @@ def prepare_layers(w, device, copies):
     return layers
 
 
-def run_ours(args, rank, world, device):
+def run_ours(args, rank, world, device, w=None):
     import bit_mixed_precision_tri_b200 as tri
-    w = workload_from_args(args.workload, args.M, args.fmt)
+    if w is None:
+        w = workload_from_args(args.workload, args.M, args.fmt)
     M, fmt = w["M"], w["fmt"]
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     step_bytes = sum(algo_bytes(fmt, M, N, K) for N, K in w["layers"])
@@ -301,6 +309,53 @@ def run_ours(args, rank, world, device):
         "clocks": clk,
     }
     return res
+
+
+def measure_cublas_fp16(w, device, steps, warmup):
+    """The same layer sequence as a dense fp16 GEMM (torch.matmul -> cuBLAS),
+    timed the same way (one CUDA graph of K steps over rotating weight copies
+    larger than L2).  Context for the ternary path, not part of it."""
+    M = w["M"]
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    dense_bytes = sum(2 * N * K for N, K in w["layers"])
+    copies = max(2, int(np.ceil(3 * l2 / dense_bytes)) + 1)
+    g = torch.Generator(device="cpu").manual_seed(1234)
+    mats = [[(torch.randn(N, K, generator=g) * 0.02).half().to(device) for N, K in w["layers"]]]
+    for _ in range(copies - 1):
+        mats.append([t.clone() for t in mats[0]])
+    xs = [torch.randn(M, K, generator=g).half().to(device) for _, K in w["layers"]]
+    ys = [torch.empty(M, N, dtype=torch.float16, device=device) for N, _ in w["layers"]]
+    stream = torch.cuda.Stream(device)
+
+    def step(c):
+        for i in range(len(w["layers"])):
+            torch.matmul(xs[i], mats[c][i].t(), out=ys[i])
+
+    with torch.cuda.stream(stream):
+        for c in range(2):
+            step(c)
+    torch.cuda.synchronize(device)
+    gw, gs = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw, stream=stream):
+        for i in range(warmup):
+            step(i % copies)
+    with torch.cuda.graph(gs, stream=stream):
+        for i in range(steps):
+            step(i % copies)
+    gw.replay()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        gs.replay()
+        t1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1) / steps
+    bytes_step = dense_bytes + sum(2 * M * K + 2 * M * N for N, K in w["layers"])
+    del gw, gs, mats
+    return {"ms_per_step": ms, "GB/s": bytes_step / (ms * 1e-3) / 1e9,
+            "TFLOP/s": sum(2.0 * M * N * K for N, K in w["layers"]) / (ms * 1e-3) / 1e12,
+            "weight_copies": copies}
 
 
 # ------------------------------------------------------------------ other rows
@@ -433,6 +488,40 @@ def allreduce_max(x, world, device):
     return float(t.item())
 
 
+SWEEP_M = [1, 2, 4, 8, 16, 32, 64, 128, 256, 512]
+
+
+def run_sweep(args, rank, world, device):
+    """Batch sweep on W 8192x8192 (TQ2 and TQ1), the 70B-like block at M = 16
+    and the format stress set on W 14336x4096 (P(0) in {0.3, 0.5, 0.7, 0.9},
+    per-block scales, M in {1, 16, 128}); one JSON line each, with the cuBLAS
+    fp16 time of the same shapes beside it."""
+    jobs = []
+    for fmt in ("tq2", "tq1"):
+        for M in SWEEP_M:
+            jobs.append(dict(name=f"sweep_8192_{fmt}_m{M}", layers=[(8192, 8192)], M=M, fmt=fmt, seeds=[5]))
+    jobs.append(dict(WORKLOADS["block70b_m16"], name="block70b_m16"))
+    for fmt in ("tq2", "tq1"):
+        for p0 in (0.3, 0.5, 0.7, 0.9):
+            for M in (1, 16, 128):
+                jobs.append(dict(name=f"stress_14336x4096_{fmt}_p{p0}_m{M}", layers=[(14336, 4096)], M=M,
+                                 fmt=fmt, seeds=[20 + int(10 * p0)], p_zero=p0))
+    cublas_cache = {}
+    for job in jobs:
+        a = argparse.Namespace(**vars(args))
+        a.steps, a.warmup = min(args.steps, 10), max(3, min(args.warmup, 3))
+        res = run_ours(a, rank, world, device, w=job)
+        key = (tuple(job["layers"]), job["M"])
+        if not args.no_cublas:
+            if key not in cublas_cache:
+                cublas_cache[key] = measure_cublas_fp16(job, device, a.steps, a.warmup)
+            cb = dict(cublas_cache[key])
+            cb["speedup_of_ternary"] = cb["ms_per_step"] / res["ms_per_step"]
+            res["cublas_fp16"] = cb
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -444,6 +533,9 @@ def main():
     ap.add_argument("--fmt", default=None, choices=[None, "tq2", "tq1"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip timing the offline rows")
+    ap.add_argument("--no-cublas", action="store_true", help="skip the cuBLAS fp16 comparison")
+    ap.add_argument("--sweep", action="store_true",
+                    help="print one line per batch-sweep, block and format-stress workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -464,7 +556,15 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=device)
     try:
+        if args.sweep:
+            run_sweep(args, rank, world, device)
+            return
         res = run_ours(args, rank, world, device)
+        if not args.no_cublas:
+            w = workload_from_args(args.workload, args.M, args.fmt)
+            cb = measure_cublas_fp16(w, device, args.steps, args.warmup)
+            cb["speedup_of_ternary"] = cb["ms_per_step"] / res["ms_per_step"]
+            res["cublas_fp16"] = cb
         if not args.no_rows:
             res["rows"] = measure_rows(device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
