@@ -31,7 +31,8 @@
 //  * Streaming.  Work = (128-row tile) x (pair of blocks) units split over a
 //    persistent grid as contiguous ranges (stream-K): every CTA streams the
 //    same number of weight bytes.  Each warp owns 16 rows of the tile and
-//    keeps four units of 16-byte cp.async copies in flight.  A row tile split
+//    keeps four units of 16-byte cp.async copies in flight, the first four
+//    copied before the wait for the preceding grid.  A row tile split
 //    between CTAs is summed, in CTA order (deterministic), by the CTA that
 //    holds its first unit; the others leave partial sums stamped with the
 //    call's epoch (one 64-bit store each: no fence, no atomic).  The epoch is
@@ -206,14 +207,17 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
     }
     if (commit) cp_async_commit();                    // one group per stage (empty at the end)
   };
-  // The weights do not depend on X: the first stage is copied before waiting
-  // for the grid that produced X (programmatic dependent launch).  Every CTA
-  // lets the next grid launch as soon as it runs: that grid can only start
-  // once all CTAs of this one have done so, i.e. are resident, so its CTAs
-  // never take a slot that a CTA of this grid (which a reducer may wait for)
-  // still needs.
+  // The weights do not depend on X: the whole ring is copied before waiting
+  // for the grid that produced X (programmatic dependent launch), so a CTA
+  // that launched early has its first weights in place when the wait ends.
+  // (Kernels that write qs or d must therefore not let this one launch early;
+  // none of this library's do.)  Every CTA lets the next grid launch as soon
+  // as it runs: that grid can only start once all CTAs of this one have done
+  // so, i.e. are resident, so its CTAs never take a slot that a CTA of this
+  // grid (which a reducer may wait for) still needs.
   ptx::griddep_launch_dependents();
-  issue(0, true);                                     // group 0: weight stage 0
+#pragma unroll
+  for (int st = 0; st < S; ++st) issue(st, true);     // group s: weight stage s
   ptx::griddep_wait();
   // this call's stamp: epoch and slot (the previous grid's epoch update is visible now)
   const unsigned long long stamp =
@@ -230,8 +234,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
     // i.e. word L/2 of the block, bytes 2(L&1) and 2(L&1)+1, fields 0..3: the
     // two bytes of field g land in one 16-bit half of fragment register
     // (p, g, r) of the thread with threadID_in_group = tig.  The X loads of up
-    // to four blocks per warp are in flight together, ahead of weight stages
-    // 1..S-1.
+    // to four blocks per warp are in flight together.
     const int f_word = lane >> 1, half = lane & 1;
     const int f_tig = f_word >> 2, f_p = (f_word >> 1) & 1, f_r = f_word & 1;
     constexpr int kXB = 4;
@@ -250,10 +253,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
                           ? __ldg(reinterpret_cast<const uint4*>(p.X + (size_t)m * p.K + (size_t)blk * kBlock) + lane)
                           : make_uint4(0, 0, 0, 0);
       }
-      if (hb0 == warp) {
-#pragma unroll
-        for (int st = 1; st < S; ++st) issue(st, true);
-      }
+
 #pragma unroll
       for (int x = 0; x < kXB; ++x) {
         const int hb = hb0 + x * kWarps;
@@ -317,10 +317,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
         }
       }
     }
-    if (warp >= n_blk) {                              // warps without a block still issue their stages
-#pragma unroll
-      for (int st = 1; st < S; ++st) issue(st, true);
-    }
+
   }
   __syncthreads();                                    // fragments visible to every warp
 
@@ -515,10 +512,13 @@ Layout layout_m(int64_t N, int64_t K, int num_sms) {
   L.P = (int)ceil_div(B, 2);
   L.T = (int)ceil_div(N, kRT);
   L.U = (long long)L.T * L.P;
-  // at least two units per CTA, at most two CTAs per SM, and few enough units
-  // per CTA that its block pairs fit in shared memory
+  // at least two units per CTA and few enough that the CTA's block pairs fit
+  // in shared memory; one CTA per SM while the work is small (up to eight
+  // units per SM), so that consecutive calls' CTAs share the SMs and the next
+  // call's prologue overlaps this one, else two per SM
   long long G = L.U / 2;
-  if (G > 2LL * num_sms) G = 2LL * num_sms;
+  const long long per_sm = L.U <= 8LL * num_sms ? 1 : 2;
+  if (G > per_sm * num_sms) G = per_sm * num_sms;
   if (G < 1) G = 1;
   if (ceil_div(L.U, G) > C::kMaxPairs) G = ceil_div(L.U, C::kMaxPairs);
   L.G = (int)G;
