@@ -101,8 +101,15 @@ def unpack(qs: torch.Tensor, N: int, K: int, fmt="tq2", return_invalid: bool = F
 
 
 # ------------------------------------------------------------------ a6
+_WS_BYTES = {}
+
+
 def gemm_workspace_bytes(fmt, M: int, N: int, K: int) -> int:
-    return int(_lib.lib().tri_gemm_workspace_bytes(_fmt(fmt), M, N, K))
+    key = (_fmt(fmt), M, N, K, torch.cuda.current_device() if torch.cuda.is_available() else -1)
+    v = _WS_BYTES.get(key)
+    if v is None:
+        v = _WS_BYTES[key] = int(_lib.lib().tri_gemm_workspace_bytes(key[0], M, N, K))
+    return v
 
 
 def auto_path(fmt, M: int, N: int, K: int) -> int:
@@ -137,16 +144,27 @@ def gemm(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, N: int, K: int, fmt
          path: int = PATH_AUTO, out: torch.Tensor = None, workspace: Workspace = None,
          stream=None) -> torch.Tensor:
     """Y = X (d * W_hat)^T in fp16 with fp32 accumulation."""
-    _require_cuda(X, qs, d)
+    # the checks a decode step pays on every call, kept to attribute reads
+    if not (X.is_cuda and qs.is_cuda and d.is_cuda):
+        raise ValueError("tensors must live on a CUDA device")
+    if not (X.is_contiguous() and qs.is_contiguous() and d.is_contiguous()):
+        raise ValueError("tensors must be contiguous")
     if X.dtype != torch.float16:
         raise ValueError("X must be float16")
     M = X.shape[0]
-    f = _fmt(fmt)
-    Y = out if out is not None else torch.empty(M, N, dtype=torch.float16, device=X.device)
+    f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+    if out is None:
+        Y = torch.empty(M, N, dtype=torch.float16, device=X.device)
+    else:
+        if not (out.is_cuda and out.is_contiguous()):
+            raise ValueError("out must be a contiguous CUDA tensor")
+        Y = out
     ws = (workspace or _workspace_for(X.device)).get(gemm_workspace_bytes(f, M, N, K))
     s = stream.cuda_stream if stream is not None else _stream(X.device)
-    _lib.check(_lib.lib().tri_gemm(f, int(path), _ptr(X), _ptr(qs), _ptr(d), _ptr(Y), M, N, K,
-                                   _ptr(ws), ws.numel(), s), "tri_gemm")
+    st = _lib.lib().tri_gemm(f, int(path), X.data_ptr(), qs.data_ptr(), d.data_ptr(), Y.data_ptr(),
+                             M, N, K, ws.data_ptr(), ws.numel(), s)
+    if st:
+        _lib.check(st, "tri_gemm")
     return Y
 
 

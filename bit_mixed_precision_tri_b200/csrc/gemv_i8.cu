@@ -632,10 +632,16 @@ cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half
 // (every CTA of the grid must be resident at once: reducers wait for others).
 bool gemv_i8_supported(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || M > 2 || N < 1 || K < kBlock || K % kBlock) return false;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
-    return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  static std::once_flag once[kMaxDev];
+  static int sm_count[kMaxDev];
+  std::call_once(once[dev], [dev]() {
+    if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sm_count[dev] = 0;
+  });
+  const int sms = sm_count[dev];
+  if (sms < 1) return false;
   const Layout L = layout_for(M, N, K, sms);
   return L.G <= 2LL * sms;
 }
