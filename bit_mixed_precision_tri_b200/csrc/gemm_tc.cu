@@ -5,29 +5,31 @@
 // enough that arithmetic, not weight traffic, bounds the layer (section
 // "TriRun: ternary inference on GPUs": the speedup falls once the product
 // becomes compute-bound).  The pages' kernel used mma.sync; this one uses the
-// fifth-generation tensor cores:
+// fifth-generation tensor cores with the decoded weights in tensor memory,
+// computing the transposed product Y^T = (d * W_hat) X^T tile by tile:
 //
-//  * a producer thread TMA-loads, per 64-wide K step, the activation tile
-//    (128 rows x 64 fp16, 128-byte swizzle) and the packed weight tile
-//    (BN rows x 16 bytes) into a ring of mbarrier-tracked stages;
-//  * BN/32 decoder warps (one weight row per thread) turn sixteen 2-bit
-//    fields per 32-bit word into exact fp16 values t * d (mask + OR with an
-//    fp16 exponent, subtract the bias, multiply by the block scale) and
-//    store them as the K-major, 128-byte-swizzled B operand;
-//  * one thread issues tcgen05.mma (M = 128, N = BN, K = 16, fp32 accumulate)
-//    with both operands in shared memory and the accumulator in tensor
-//    memory, and frees stages with tcgen05.commit;
-//  * the decoder warps finally read the accumulator with tcgen05.ld and
-//    write fp16 Y (or fp32 partials when K is split across CTAs; the last
-//    CTA of a tile sums them in split order, so results are deterministic).
-//
-// The decode emits the pairs (w_j, w_{j+8}) of each 16-weight word, so the
-// activations are consumed in the same within-16 order: a prep kernel writes
-// X once per call in that order (pairs (x_j, x_{j+8}) adjacent) and zeroes
-// the split-K tickets; it is chained to the main kernel with programmatic
-// dependent launch.
-#include <cstdlib>
-
+//  * a tile is 128 weight rows (the MMA's M, one TMEM lane per row) by NB <= 256
+//    activation rows (the MMA's N); its K range may be split over the CTAs of
+//    a thread-block cluster;
+//  * two producer threads TMA-load, per 64-wide K step, the activation tile
+//    (NB rows x 64 fp16, 128-byte swizzle) straight from X; a third loads the
+//    packed weights one 256-wide block at a time (128 rows x 64 B, 64-byte
+//    swizzle).  A single issuing thread is latency-bound near one TMA load per
+//    ~300 cycles, so the loads are spread over threads;
+//  * eight decoder warps (two per TMEM lane quarter, one K half each) turn
+//    each byte's four 2-bit fields into two fp16 pairs (w_k, w_k+1) = t * d in
+//    natural K order (byte spread + mask + OR with fp16 exponents, subtract the
+//    bias, multiply by the block scale -- all exact) and store them into a
+//    ring of A slots in tensor memory with tcgen05.st, so the decoded weights
+//    never touch shared memory and X needs no reordering;
+//  * one thread issues tcgen05.mma (M = 128, N = NB, K = 16, fp32 accumulate)
+//    with A in tensor memory and the activations in shared memory; a stage's
+//    commit frees both its activation buffer and its A slot;
+//  * the epilogue reads the accumulator with tcgen05.ld.  When K is split, the
+//    CTAs of the cluster send each other 32-column slices of their partial
+//    sums through distributed shared memory; each slice's owner adds the
+//    partials in cluster-rank order, so results are deterministic.  No global
+//    scratch and no inter-CTA tickets are involved.
 #include <cudaTypedefs.h>
 
 #include "sm100_ptx.cuh"
@@ -36,98 +38,103 @@
 namespace tri {
 namespace {
 
-constexpr int BM = 128;   // activation rows per tile (MMA M)
-constexpr int BK = 64;    // K per stage: one 128-byte swizzle row of fp16
+constexpr int kRows = 128;                        // weight rows per tile (MMA M, TMEM lanes)
+constexpr int BK = 64;                            // K per MMA stage: one 128-byte swizzle row
+constexpr int kStepsPerBlock = kBlock / BK;       // 4
+constexpr int kPBytes = kRows * (kBlock / 4);     // packed block tile: 8 KB
+constexpr int kPStages = 4;
+constexpr int kMaxStages = 8;                     // activation stages = A slots
+constexpr int kAColBase = 256;                    // A slots live after the accumulator columns
+constexpr int kACols = BK / 2;                    // 64 fp16 per lane = 32 columns
+constexpr int kFirstDec = 4;                      // warps 0,2: X producers; 1: MMA; 3: P producer
+constexpr int kDecWarps = 8;
+constexpr int kThreads = (kFirstDec + kDecWarps) * 32;
+constexpr int kRingBudget = 192 * 1024;
+constexpr int kMinSmem = 120 * 1024;              // > half an SM: one CTA (and TMEM owner) per SM
+constexpr int kRecvStride = 36;                   // floats per staged row slice (32 + pad)
+constexpr int kChunkBytes = kRows * kRecvStride * 4;  // one 32-column slice of a partial tile
+
+// most chunks a rank sends (it owns at least floor(nch / sp) of the nch chunks)
+__host__ __device__ constexpr int max_out_chunks(int nch, int sp) { return nch - nch / sp; }
+__host__ __device__ constexpr int max_own_chunks(int nch, int sp) { return (nch + sp - 1) / sp; }
 constexpr uint32_t kWaitLimit = 1u << 22;
 
-template <int BN>
-struct Cfg {
-  static constexpr int DW = BN / 32;                 // decoder / epilogue warps
-  static constexpr int kThreads = (2 + DW) * 32;
-  static constexpr int kXBytes = BM * BK * 2;        // 16 KB
-  static constexpr int kDBytes = BN * BK * 2;        // decoded fp16 weight tile
-  static constexpr int kPBytes = BN * BK / 4;        // packed 2-bit weight tile
-  static constexpr int kStages = (BN == 256) ? 4 : 6;
-  static constexpr int kSmem = kStages * (kXBytes + kDBytes + kPBytes) + 1024 + 512;
-};
-
 struct TcParams {
-  float* partials;      // [tiles][splits][BM][BN]
-  unsigned* counters;   // [tiles]
   unsigned* error;
-  int M, N, K, B, ksteps, splits, tiles_n;
+  int M, N, K, B;      // B = K / 256 blocks
+  int NB;              // activation rows per tile (MMA N)
+  int S;               // activation stages (even, <= kMaxStages)
+  int splits;          // CTAs per cluster sharing one tile's K range
 };
 
-// ---------------------------------------------------------------- prep kernel
-__global__ void __launch_bounds__(256)
-xperm_kernel(const __half* __restrict__ X, int64_t groups, __half* __restrict__ Xp,
-             unsigned* __restrict__ tickets, int ntickets) {
-  ptx::griddep_launch_dependents();
-  if (blockIdx.x == 0)    // split-K tickets start at zero on every call
-    for (int i = threadIdx.x; i < ntickets; i += blockDim.x) tickets[i] = 0u;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < groups; i += stride) {
-    const uint4* src = reinterpret_cast<const uint4*>(X) + 2 * i;
-    const uint4 lo = src[0], hi = src[1];
-    const uint32_t lw[4] = {lo.x, lo.y, lo.z, lo.w}, hw[4] = {hi.x, hi.y, hi.z, hi.w};
-    uint32_t pr[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) pr[j] = __byte_perm(lw[j >> 1], hw[j >> 1], (j & 1) ? 0x7632 : 0x5410);
-    uint4* dst = reinterpret_cast<uint4*>(Xp) + 2 * i;
-    dst[0] = make_uint4(pr[0], pr[1], pr[2], pr[3]);
-    dst[1] = make_uint4(pr[4], pr[5], pr[6], pr[7]);
-  }
+size_t smem_bytes(int NB, int S) {
+  const size_t need = 1024 + (size_t)S * NB * 128 + (size_t)kPStages * kPBytes +
+                      (2 * kMaxStages + 2 * kPStages + 2) * 8 + 16;
+  return need < (size_t)kMinSmem ? (size_t)kMinSmem : need;
 }
 
-// (beta_j + d') pair from field position j of both halves, then exact t * d
-__device__ __forceinline__ uint32_t decode_scaled(uint32_t w, int j, __half2 dd) {
-  const uint32_t mask = 0x00030003u << (2 * j);
-  const uint32_t e = (j == 0) ? 0x6400u : (j == 1) ? 0x5C00u : (j == 2) ? 0x5400u : 0x4C00u;
-  const uint32_t b1 = (j == 0) ? 0x6401u : (j == 1) ? 0x5C04u : (j == 2) ? 0x5410u : 0x4C40u;
-  const uint32_t h = (w & mask) | (e | (e << 16));
-  __half2 hv = *reinterpret_cast<const __half2*>(&h);
-  const uint32_t bb = b1 | (b1 << 16);
-  const __half2 bias = *reinterpret_cast<const __half2*>(&bb);
-  __half2 t = __hsub2(hv, bias);          // exactly d' - 1
-  t = __hmul2(t, dd);                     // exactly t * d
+// Two fp16 weights (w_k, w_k+1) of one byte (spread into both 16-bit halves):
+// field 2f in the low half, field 2f+1 in the high half, each read as the low
+// mantissa bits of an fp16 constant, minus (constant + 1) gives the trit
+// exactly; times the block scale gives t * d exactly.
+template <int F>
+__device__ __forceinline__ uint32_t pair_of(uint32_t spread, __half2 dd) {
+  constexpr uint32_t mask = F == 0 ? 0x000C0003u : 0x00C00030u;
+  constexpr uint32_t expo = F == 0 ? 0x5C006400u : 0x4C005400u;   // 256 | 1024, 16 | 64
+  constexpr uint32_t bias = F == 0 ? 0x5C046401u : 0x4C405410u;   // 257 | 1025, 17 | 65
+  const uint32_t h = (spread & mask) | expo;
+  const uint32_t b = bias;
+  __half2 t = __hsub2(*reinterpret_cast<const __half2*>(&h), *reinterpret_cast<const __half2*>(&b));
+  t = __hmul2(t, dd);
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
-template <int BN>
-__global__ void __launch_bounds__(Cfg<BN>::kThreads, 1)
+__device__ __forceinline__ void store_y(__half* __restrict__ Y, const uint32_t (&v)[32], int n,
+                                        int mbase, int lim, int N) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e)
+    if (e < lim) Y[(size_t)(mbase + e) * N + n] = __float2half_rn(__uint_as_float(v[e]));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap qmap,
                const __half* __restrict__ dsc, __half* __restrict__ Y, const TcParams p) {
-  using C = Cfg<BN>;
-  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* xs = smem;                                   // S x kXBytes (1024-aligned)
-  uint8_t* ds = xs + S * C::kXBytes;                    // S x kDBytes (1024-aligned)
-  uint8_t* ps = ds + S * C::kDBytes;                    // S x kPBytes
-  uint64_t* full = reinterpret_cast<uint64_t*>(ps + S * C::kPBytes);
-  uint64_t* dec = full + S;
-  uint64_t* empty = dec + S;
-  uint64_t* accf = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
-  volatile int* s_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int S = p.S, NB = p.NB;
+  const uint32_t XB = (uint32_t)NB * 128;
+  uint8_t* xs = smem;                                            // S x XB (1024-aligned)
+  uint8_t* ps = xs + (size_t)S * XB;                             // kPStages x kPBytes
+  uint64_t* full = reinterpret_cast<uint64_t*>(ps + kPStages * kPBytes);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* pfull = empty + kMaxStages;
+  uint64_t* pempty = pfull + kPStages;
+  uint64_t* accf = pempty + kPStages;
+  uint64_t* recvf = accf + 1;                                    // split-K slices received
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recvf + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
-  const int ks0 = (int)((int64_t)p.ksteps * split / p.splits);
-  const int ks1 = (int)((int64_t)p.ksteps * (split + 1) / p.splits);
-  const int nks = ks1 - ks0;
+  const int b0 = (int)((int64_t)p.B * split / p.splits);
+  const int nblk = (int)((int64_t)p.B * (split + 1) / p.splits) - b0;
+  const int nks = nblk * kStepsPerBlock;
 
+  ptx::griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(&full[s], 1);
-      ptx::mbar_init(&dec[s], C::DW);
-      ptx::mbar_init(&empty[s], 1);
+      ptx::mbar_init(&full[s], kDecWarps + 1);     // 8 decoder warps + the X producer (with tx)
+      ptx::mbar_init(&empty[s], 1);                // MMA commit
+    }
+    for (int s = 0; s < kPStages; ++s) {
+      ptx::mbar_init(&pfull[s], 1);
+      ptx::mbar_init(&pempty[s], kDecWarps);
     }
     ptx::mbar_init(accf, 1);
+    ptx::mbar_init(recvf, 1);
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_slot, BN);
+    ptx::tmem_alloc(tmem_slot, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -135,208 +142,222 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      ptx::prefetch_tensormap(&xmap);
-      ptx::prefetch_tensormap(&qmap);
-      const uint64_t pol_w = ptx::policy_evict_first();
-      uint64_t pol_x;
-      asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_x));
-      uint32_t limit = kWaitLimit;
-      ptx::griddep_wait();      // activations are written by the prep kernel
-      for (int i = 0; i < nks; ++i) {
-        const int s = i % S;
-        const uint32_t ph = (uint32_t)((i / S) & 1);
-        if (i >= S && !ptx::mbar_wait(&empty[s], ph ^ 1u, limit)) {
-          atomicExch(p.error, 11u);
-          limit = 1;
-        }
-        const int ks = ks0 + i;
-        ptx::mbar_arrive_expect_tx(&full[s], C::kXBytes + C::kPBytes);
-        ptx::tma_load_2d(xs + s * C::kXBytes, &xmap, ks * BK, m_tile * BM, &full[s], pol_x);
-        ptx::tma_load_2d(ps + s * C::kPBytes, &qmap, ks * (BK / 4), n_tile * BN, &full[s], pol_w);
+  // decoder / epilogue geometry (meaningful for warps >= kFirstDec)
+  const int q = warp & 3, h = (warp - kFirstDec) >> 2;
+  const int r = 32 * q + lane;                         // weight row in the tile = TMEM lane
+  const int n = n_tile * kRows + r;
+  const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
+  uint32_t limit = kWaitLimit;
+
+  if ((warp == 0 || warp == 2) && lane == 0) {
+    // -------------------------------------------------- activation producers
+    ptx::prefetch_tensormap(&xmap);
+    uint64_t pol_x;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_x));
+    ptx::griddep_wait();           // X may be the previous kernel's output
+    int s = warp >> 1, round = 0;
+    for (int i = warp >> 1; i < nks; i += 2) {
+      if (round > 0 && !ptx::mbar_wait(&empty[s], (uint32_t)((round - 1) & 1), limit)) {
+        atomicExch(p.error, 21u);
+        limit = 1;
       }
+      ptx::mbar_arrive_expect_tx(&full[s], XB);
+      ptx::tma_load_2d(xs + (size_t)s * XB, &xmap, (b0 * kStepsPerBlock + i) * BK, m_tile * NB,
+                       &full[s], pol_x);
+      s += 2;
+      if (s >= S) { s -= S; ++round; }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = (1u << 4)                  // D: f32
-                             | ((uint32_t)(BN >> 3) << 17)  // N
-                             | ((uint32_t)(BM >> 4) << 24); // M ; A, B: f16, K-major
-      uint32_t limit = kWaitLimit;
-      for (int i = 0; i < nks; ++i) {
-        const int s = i % S;
-        const uint32_t ph = (uint32_t)((i / S) & 1);
-        if (!ptx::mbar_wait(&dec[s], ph, limit) || !ptx::mbar_wait(&full[s], ph, limit)) {
-          atomicExch(p.error, 12u);
+  } else if (warp == 3 && lane == 0) {
+    // -------------------------------------------------- packed weight producer
+    ptx::prefetch_tensormap(&qmap);
+    const uint64_t pol_w = ptx::policy_evict_first();
+    int s = 0;
+    uint32_t ph = 0;
+    for (int j = 0; j < nblk; ++j) {
+      if (j >= kPStages && !ptx::mbar_wait(&pempty[s], ph ^ 1u, limit)) {
+        atomicExch(p.error, 22u);
+        limit = 1;
+      }
+      ptx::mbar_arrive_expect_tx(&pfull[s], kPBytes);
+      ptx::tma_load_2d(ps + s * kPBytes, &qmap, (b0 + j) * (kBlock / 4), n_tile * kRows, &pfull[s], pol_w);
+      if (++s == kPStages) { s = 0; ph ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // -------------------------------------------------- MMA issuer
+    const uint32_t idesc = (1u << 4)                        // D: f32
+                           | ((uint32_t)(NB >> 3) << 17)     // N
+                           | ((uint32_t)(kRows >> 4) << 24); // M = 128; A, B: f16, K-major
+    const uint32_t xs_u = ptx::smem_u32(xs);
+    int s = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < nks; ++i) {
+      if (!ptx::mbar_wait(&full[s], ph, limit)) {
+        atomicExch(p.error, 23u);
+        limit = 1;
+      }
+      ptx::tc_fence_after();
+      const uint64_t bdesc = ptx::sw128_kmajor_desc(xs_u + (uint32_t)s * XB);
+      const uint32_t a_tm = tmem + (uint32_t)(kAColBase + s * kACols);
+#pragma unroll
+      for (int k = 0; k < BK / 16; ++k)
+        ptx::umma_f16_ts(tmem, a_tm + (uint32_t)(8 * k), bdesc + (uint64_t)(2 * k), idesc,
+                         (i > 0 || k > 0) ? 1u : 0u);
+      ptx::umma_commit(&empty[s]);
+      if (++s == S) { s = 0; ph ^= 1u; }
+    }
+    ptx::umma_commit(accf);
+  } else if (warp >= kFirstDec) {
+    // -------------------------------------------------- decoders
+    const bool nvalid = n < p.N;
+    const __half* drow = dsc + (size_t)(nvalid ? n : 0) * p.B + b0;
+    const uint32_t ps_u = ptx::smem_u32(ps);
+    // this thread's 8 bytes of K step t: 16-byte granule t of row r, 64-byte swizzle, half h
+    const uint32_t row_off = (uint32_t)(r * 64 + 8 * h);
+    const uint32_t swz = (uint32_t)((r >> 1) & 3);
+    __half dnext = nvalid ? __ldg(drow) : __float2half(0.f);
+    int s = 0, round = 0, pst = 0;
+    uint32_t pph = 0;
+    for (int j = 0; j < nblk; ++j) {
+      const __half2 dd = __halves2half2(dnext, dnext);
+      if (j + 1 < nblk) dnext = nvalid ? __ldg(drow + j + 1) : __float2half(0.f);
+      if (!ptx::mbar_wait(&pfull[pst], pph, limit)) {
+        atomicExch(p.error, 24u);
+        limit = 1;
+      }
+      uint2 wv[kStepsPerBlock];
+      const uint32_t pbase = ps_u + (uint32_t)(pst * kPBytes) + row_off;
+#pragma unroll
+      for (int t = 0; t < kStepsPerBlock; ++t) wv[t] = ptx::lds64(pbase + ((((uint32_t)t) ^ swz) << 4));
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&pempty[pst]);
+      if (++pst == kPStages) { pst = 0; pph ^= 1u; }
+#pragma unroll
+      for (int t = 0; t < kStepsPerBlock; ++t) {
+        if (round > 0 && !ptx::mbar_wait(&empty[s], (uint32_t)((round - 1) & 1), limit)) {
+          atomicExch(p.error, 25u);
           limit = 1;
         }
         ptx::tc_fence_after();
-        const uint64_t a0 = ptx::sw128_kmajor_desc(ptx::smem_u32(xs + s * C::kXBytes));
-        const uint64_t b0 = ptx::sw128_kmajor_desc(ptx::smem_u32(ds + s * C::kDBytes));
+        __syncwarp();                    // tcgen05.st below is warp-collective
+        uint32_t a[16];
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          ptx::umma_f16_ss(tmem, a0 + 2 * k, b0 + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
-        ptx::umma_commit(&empty[s]);
+        for (int b = 0; b < 8; ++b) {
+          const uint32_t w = b < 4 ? wv[t].x : wv[t].y;
+          const uint32_t sel = (uint32_t)(b & 3) * 0x0101u + 0x4040u;   // byte b into both halves
+          const uint32_t spread = __byte_perm(w, 0u, sel);
+          a[2 * b] = pair_of<0>(spread, dd);
+          a[2 * b + 1] = pair_of<1>(spread, dd);
+        }
+        ptx::tmem_st_32x32b_x16(lane_base + (uint32_t)(kAColBase + s * kACols + 16 * h), a);
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&full[s]);
+        if (++s == S) { s = 0; ++round; }
       }
-      ptx::umma_commit(accf);
     }
-  } else {
-    // ------------------------------------------------------------ decoders
-    const int r = (warp - 2) * 32 + lane;            // weight row within the tile
-    const int n = n_tile * BN + r;
-    const uint32_t ps_u = ptx::smem_u32(ps), ds_u = ptx::smem_u32(ds);
-    uint32_t limit = kWaitLimit;
-    __half2 dd = __float2half2_rn(0.f);
-    for (int i = 0; i < nks; ++i) {
-      const int s = i % S;
-      const uint32_t ph = (uint32_t)((i / S) & 1);
-      const int ks = ks0 + i;
-      if (i == 0 || (ks & 3) == 0) {
-        const __half dv = n < p.N ? __ldg(dsc + (size_t)n * p.B + (ks >> 2)) : __float2half(0.f);
-        dd = __halves2half2(dv, dv);
-      }
-      if (!ptx::mbar_wait(&full[s], ph, limit)) {
-        atomicExch(p.error, 13u);
-        limit = 1;
-      }
-      const uint4 pw = ptx::lds128(ps_u + (uint32_t)(s * C::kPBytes + r * 16));
-      const uint32_t w4[4] = {pw.x, pw.y, pw.z, pw.w};
-      const uint32_t row_base = ds_u + (uint32_t)(s * C::kDBytes + r * 128);
+    if (!ptx::mbar_wait(accf, 0, limit)) atomicExch(p.error, 26u);
+    ptx::tc_fence_after();
+    __syncwarp();
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  const int nch = (NB + 31) / 32;                      // 32-column accumulator chunks
+  const bool dec = warp >= kFirstDec;
+  const int mtile0 = m_tile * NB;
+  if (p.splits > 1) {
+    // Split K: chunk c of the accumulator belongs to rank c % sp.  Each CTA
+    // stages the chunks it does not own in its (now idle) rings, then one
+    // thread bulk-copies each to its owner; owners add the slices in rank order.
+    const int sp = p.splits;
+    const uint32_t area = ptx::smem_u32(xs);
+    const int nown = split < nch ? (nch - 1 - split) / sp + 1 : 0;
+    const uint32_t recv0 = (uint32_t)(max_out_chunks(nch, sp) * kChunkBytes);
+    if (dec) {
+      for (int c = h; c < nch; c += 2) {
+        if (c % sp == split) continue;
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(32 * c), v);
+        ptx::tmem_ld_wait();
+        const int before = c > split ? (c - split + sp - 1) / sp : 0;    // owned chunks below c
+        const uint32_t row = area + (uint32_t)((c - before) * kChunkBytes + r * kRecvStride * 4);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t w = w4[q], wsh = w >> 8;
-        const int c0 = (2 * q) ^ (r & 7), c1 = (2 * q + 1) ^ (r & 7);
-        ptx::sts128(row_base + c0 * 16, decode_scaled(w, 0, dd), decode_scaled(w, 1, dd),
-                    decode_scaled(w, 2, dd), decode_scaled(w, 3, dd));
-        ptx::sts128(row_base + c1 * 16, decode_scaled(wsh, 0, dd), decode_scaled(wsh, 1, dd),
-                    decode_scaled(wsh, 2, dd), decode_scaled(wsh, 3, dd));
+        for (int g = 0; g < 8; ++g) ptx::sts128u(row + 16u * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
       }
       ptx::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&dec[s]);
     }
-    // ------------------------------------------------------------ epilogue
-    if (!ptx::mbar_wait(accf, 0, limit)) atomicExch(p.error, 14u);
-    ptx::tc_fence_after();
-    const int quarter = warp & 3;
-    constexpr int kColsPerWarp = BN / (C::DW / 4);
-    const int col_base = ((warp - 2) / 4) * kColsPerWarp;
-    const int m = m_tile * BM + 32 * quarter + lane;
-    const int tile = m_tile * p.tiles_n + n_tile;
-    for (int j = 0; j < kColsPerWarp / 32; ++j) {
-      const int col0 = col_base + 32 * j;
+    if (threadIdx.x == 0)
+      ptx::mbar_arrive_expect_tx(recvf, (uint32_t)(nown * (sp - 1) * kChunkBytes));
+    ptx::cluster_sync();               // staged slices written; every receive area is idle
+    if (threadIdx.x == 0) {
+      int o = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int owner = c % sp;
+        if (owner == split) continue;
+        const int slot = (c / sp) * (sp - 1) + (split < owner ? split : split - 1);
+        ptx::bulk_s2peer(ptx::mapa(area + recv0 + (uint32_t)(slot * kChunkBytes), (uint32_t)owner),
+                         area + (uint32_t)(o * kChunkBytes), (uint32_t)kChunkBytes,
+                         ptx::mapa(ptx::smem_u32(recvf), (uint32_t)owner));
+        ++o;
+      }
+    }
+    if (dec && !ptx::mbar_wait(recvf, 0, limit)) atomicExch(p.error, 27u);
+    ptx::cluster_sync();               // every slice landed: sources may be released
+    __syncwarp();
+    if (dec) {                         // warp-uniform: tcgen05.ld is warp-collective
+      for (int lc = h; lc < nown; lc += 2) {
+        const int c = lc * sp + split;
+        uint32_t v[32];
+        ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(32 * c), v);
+        ptx::tmem_ld_wait();
+        float acc[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+        for (int src = 0; src < sp; ++src) {
+          if (src == split) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] += __uint_as_float(v[e]);
+            continue;
+          }
+          const int slot = lc * (sp - 1) + (src < split ? src : src - 1);
+          const uint32_t a = area + recv0 + (uint32_t)(slot * kChunkBytes + r * kRecvStride * 4);
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const uint4 f = ptx::lds128(a + 16u * g);
+            acc[4 * g] += __uint_as_float(f.x);
+            acc[4 * g + 1] += __uint_as_float(f.y);
+            acc[4 * g + 2] += __uint_as_float(f.z);
+            acc[4 * g + 3] += __uint_as_float(f.w);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(acc[e]);
+        const int lim = min(min(32, NB - 32 * c), p.M - (mtile0 + 32 * c));
+        if (n < p.N) store_y(Y, v, n, mtile0 + 32 * c, lim, p.N);
+      }
+    }
+  } else if (dec) {
+    for (int c = h; c < nch; c += 2) {
       uint32_t v[32];
-      ptx::tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)col0, v);
+      ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(32 * c), v);
       ptx::tmem_ld_wait();
-      const int n0 = n_tile * BN + col0;
-      if (p.splits == 1) {
-        if (m < p.M) {
-          __half* yrow = Y + (size_t)m * p.N + n0;
-          if ((p.N & 7) == 0 && n0 + 32 <= p.N) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t h[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                __half2 t = __floats2half2_rn(__uint_as_float(v[8 * q + 2 * e]),
-                                              __uint_as_float(v[8 * q + 2 * e + 1]));
-                h[e] = *reinterpret_cast<uint32_t*>(&t);
-              }
-              reinterpret_cast<uint4*>(yrow)[q] = make_uint4(h[0], h[1], h[2], h[3]);
-            }
-          } else {
-            for (int e = 0; e < 32; ++e)
-              if (n0 + e < p.N) yrow[e] = __float2half_rn(__uint_as_float(v[e]));
-          }
-        }
-      } else {
-        float* part = p.partials + (((size_t)tile * p.splits + split) * BM + 32 * quarter + lane) * BN + col0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          reinterpret_cast<float4*>(part)[q] =
-              make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-      }
-    }
-    if (p.splits > 1) {
-      __threadfence();
-      ptx::named_bar_sync(1, C::DW * 32);
-      if (warp == 2 && lane == 0) {
-        const unsigned old = atomicAdd(&p.counters[tile], 1u);
-        *s_flag = (old == (unsigned)(p.splits - 1)) ? 1 : 0;
-      }
-      ptx::named_bar_sync(1, C::DW * 32);
-      if (*s_flag) {
-        __threadfence();
-        for (int j = 0; j < kColsPerWarp / 32; ++j) {
-          const int col0 = col_base + 32 * j;
-          const int n0 = n_tile * BN + col0;
-          float acc[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) acc[e] = 0.f;
-          for (int sp = 0; sp < p.splits; ++sp) {
-            const float4* src = reinterpret_cast<const float4*>(
-                p.partials + (((size_t)tile * p.splits + sp) * BM + 32 * quarter + lane) * BN + col0);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 f = __ldcg(src + q);
-              acc[4 * q] += f.x; acc[4 * q + 1] += f.y; acc[4 * q + 2] += f.z; acc[4 * q + 3] += f.w;
-            }
-          }
-          if (m < p.M) {
-            __half* yrow = Y + (size_t)m * p.N + n0;
-            for (int e = 0; e < 32; ++e)
-              if (n0 + e < p.N) yrow[e] = __float2half_rn(acc[e]);
-          }
-        }
-        if (warp == 2 && lane == 0) p.counters[tile] = 0u;
-      }
+      const int lim = min(min(32, NB - 32 * c), p.M - (mtile0 + 32 * c));
+      if (n < p.N) store_y(Y, v, n, mtile0 + 32 * c, lim, p.N);
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, BN);
+    ptx::tmem_dealloc(tmem, 512);
   }
 }
 
 // ---------------------------------------------------------------- host side
-size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
-
 struct Plan {
-  int BN, splits, tiles_n, tiles_m;
-  size_t off_err, off_cnt, off_xp, off_part, total;
+  int NB, S, tiles_n, tiles_m, splits;
+  size_t smem;
 };
-
-Plan plan_for(int64_t M, int64_t N, int64_t K, int num_sms) {
-  Plan pl;
-  const int64_t tm = ceil_div(M, BM);
-  const int64_t t128 = tm * ceil_div(N, 128), t256 = tm * ceil_div(N, 256);
-  const char* env = std::getenv("TRI_TC_BN");
-  int bn = env ? std::atoi(env) : 0;
-  if (bn != 128 && bn != 256) bn = (t128 <= num_sms) ? 128 : 256;
-  pl.BN = bn;
-  const int64_t tiles = bn == 128 ? t128 : t256;
-  const int64_t ksteps = K / BK;
-  int64_t sp = tiles >= num_sms ? 1 : num_sms / tiles;
-  const char* envs = std::getenv("TRI_TC_SPLITS");
-  if (envs) sp = std::atoi(envs);
-  if (sp < 1) sp = 1;
-  if (sp > ksteps) sp = ksteps;
-  if (sp > 16) sp = 16;
-  pl.splits = (int)sp;
-  pl.tiles_n = (int)ceil_div(N, bn);
-  pl.tiles_m = (int)tm;
-  pl.off_err = 0;
-  pl.off_cnt = 256;
-  pl.off_xp = pl.off_cnt + up256((size_t)tiles * 4);
-  pl.off_part = pl.off_xp + up256((size_t)M * K * 2);
-  pl.total = pl.off_part + (pl.splits > 1 ? up256((size_t)tiles * pl.splits * BM * bn * 4) : 0);
-  return pl;
-}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -350,21 +371,101 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int BN>
-cudaError_t launch_bn(const Plan& pl, const __half* X, const uint8_t* qs, const __half* d, __half* Y,
-                      int M, int N, int K, void* ws, cudaStream_t s) {
-  using C = Cfg<BN>;
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  __half* Xp = reinterpret_cast<__half*>(w + pl.off_xp);
+constexpr int kMaxSmem = 232448;                  // 227 KB: the opt-in limit per block
+
+// Raise the kernel's dynamic shared memory limit to the maximum once per device.
+cudaError_t ensure_smem_attr() {
+  static bool done[16] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 16 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e == cudaSuccess && dev >= 0 && dev < 16) done[dev] = true;
+  return e;
+}
+
+// CTAs that can run at once in clusters of `sp` (one CTA per SM), per device.
+int cluster_slots(int sp, int num_sms) {
+  static int cache[16][5] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return (num_sms / sp) * sp;
+  int& slot = cache[dev][sp];
+  if (slot) return slot;
+  int clusters = 0;
+  if (ensure_smem_attr() == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, (unsigned)sp);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kMinSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = (unsigned)sp;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel, &cfg) != cudaSuccess) clusters = 0;
+  }
+  cudaGetLastError();
+  slot = clusters > 0 ? clusters * sp : (num_sms / sp) * sp;
+  return slot;
+}
+
+Plan plan_for(int64_t M, int64_t N, int64_t K, int num_sms) {
+  Plan pl;
+  pl.tiles_m = (int)ceil_div(M, 256);
+  const int64_t per = ceil_div(M, pl.tiles_m);
+  pl.NB = (int)(ceil_div(per, 16) * 16);
+  const int XB = pl.NB * 128;
+  int S = kRingBudget / XB;
+  if (S > kMaxStages) S = kMaxStages;
+  pl.S = S & ~1;
+  pl.tiles_n = (int)ceil_div(N, kRows);
+  const int64_t tiles = (int64_t)pl.tiles_n * pl.tiles_m;
+  const int64_t B = K / kBlock;
+  const int nch = (pl.NB + 31) / 32;
+  // estimated time in K-step units: waves x (steps per CTA + fixed cost)
+  double best = 0;
+  pl.splits = 1;
+  for (int sp = 1; sp <= 4; ++sp) {
+    if (sp > B) break;
+    const int64_t area = (int64_t)(max_out_chunks(nch, sp) + max_own_chunks(nch, sp) * (sp - 1)) * kChunkBytes;
+    if (sp > 1 && area > (int64_t)pl.S * XB + (int64_t)kPStages * kPBytes) continue;
+    const int64_t slots = sp == 1 ? num_sms : cluster_slots(sp, num_sms);
+    const int64_t waves = ceil_div(tiles * sp, slots);
+    const double t = (double)waves * ((double)ceil_div(B, sp) * kStepsPerBlock + (sp == 1 ? 6.0 : 9.0));
+    if (sp == 1 || t < best) {
+      best = t;
+      pl.splits = sp;
+    }
+  }
+  pl.smem = smem_bytes(pl.NB, pl.S);
+  return pl;
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int fmt, int64_t M, int64_t N, int64_t K) {
+  return fmt == TRI_TQ2 && M >= 17 && N >= 1 && K >= kBlock && K % kBlock == 0 &&
+         ceil_div(M, 256) <= 65535;
+}
+
+size_t gemm_tc_ws_bytes(int, int64_t, int64_t, int64_t, int) { return 256; }
+
+cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __half* d, __half* Y,
+                           int M, int N, int K, void* ws, int num_sms, cudaStream_t s) {
+  if (!gemm_tc_supported(fmt, M, N, K)) return cudaErrorNotSupported;
+  const Plan pl = plan_for(M, N, K, num_sms);
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMap xmap, qmap;
   {
     const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t gstr[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t box[2] = {BK, BM};
+    const cuuint32_t box[2] = {BK, (cuuint32_t)pl.NB};
     const cuuint32_t es[2] = {1, 1};
-    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, Xp, gdim, gstr, box, es,
+    if (enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half*>(X), gdim, gstr, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
@@ -372,59 +473,35 @@ cudaError_t launch_bn(const Plan& pl, const __half* X, const uint8_t* qs, const 
   {
     const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
     const cuuint64_t gstr[1] = {(cuuint64_t)(K / 4)};
-    const cuuint32_t box[2] = {BK / 4, (cuuint32_t)BN};
+    const cuuint32_t box[2] = {kBlock / 4, kRows};
     const cuuint32_t es[2] = {1, 1};
     if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(qs), gdim, gstr, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const int64_t groups = (int64_t)M * K / 16;
-  int64_t gx = ceil_div(groups, 256);
-  if (gx > 148 * 8) gx = 148 * 8;
-  xperm_kernel<<<(unsigned)gx, 256, 0, s>>>(X, groups, Xp, reinterpret_cast<unsigned*>(w + pl.off_cnt),
-                                            pl.tiles_n * pl.tiles_m);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-
   TcParams p;
-  p.partials = reinterpret_cast<float*>(w + pl.off_part);
-  p.counters = reinterpret_cast<unsigned*>(w + pl.off_cnt);
-  p.error = reinterpret_cast<unsigned*>(w + pl.off_err);
-  p.M = M; p.N = N; p.K = K; p.B = K / kBlock; p.ksteps = K / BK; p.splits = pl.splits;
-  p.tiles_n = pl.tiles_n;
-  e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  p.error = static_cast<unsigned*>(ws);
+  p.M = M; p.N = N; p.K = K; p.B = K / kBlock;
+  p.NB = pl.NB; p.S = pl.S; p.splits = pl.splits;
+  if (pl.smem > (size_t)kMaxSmem) return cudaErrorInvalidValue;
+  const cudaError_t e = ensure_smem_attr();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)pl.tiles_n, (unsigned)pl.tiles_m, (unsigned)pl.splits);
-  cfg.blockDim = dim3(C::kThreads);
-  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = (unsigned)pl.splits;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN>, xmap, qmap, d, Y, p);
-}
-
-}  // namespace
-
-bool gemm_tc_supported(int fmt, int64_t M, int64_t N, int64_t K) {
-  return fmt == TRI_TQ2 && M >= 17 && N >= 1 && K >= kBlock && K % kBlock == 0 &&
-         ceil_div(M, BM) <= 65535;
-}
-
-size_t gemm_tc_ws_bytes(int, int64_t M, int64_t N, int64_t K, int num_sms) {
-  return plan_for(M, N, K, num_sms).total;
-}
-
-cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __half* d, __half* Y,
-                           int M, int N, int K, void* ws, int num_sms, cudaStream_t s) {
-  if (!gemm_tc_supported(fmt, M, N, K)) return cudaErrorNotSupported;
-  const Plan pl = plan_for(M, N, K, num_sms);
-  if (pl.BN == 256) return launch_bn<256>(pl, X, qs, d, Y, M, N, K, ws, s);
-  return launch_bn<128>(pl, X, qs, d, Y, M, N, K, ws, s);
+  cfg.numAttrs = pl.splits > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel, xmap, qmap, d, Y, p);
 }
 
 }  // namespace tri
