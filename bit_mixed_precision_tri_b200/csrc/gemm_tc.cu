@@ -69,7 +69,7 @@ struct TcParams {
 
 size_t smem_bytes(int NB, int S) {
   const size_t need = 1024 + (size_t)S * NB * 128 + (size_t)kPStages * kPBytes +
-                      (2 * kMaxStages + 2 * kPStages + 2) * 8 + 16;
+                      (kMaxStages + 2 * kPStages + 2) * 8 + 16;
   return need < (size_t)kMinSmem ? (size_t)kMinSmem : need;
 }
 
@@ -101,13 +101,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                const __half* __restrict__ dsc, __half* __restrict__ Y, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.S, NB = p.NB;
+  const int S = p.S, NB = p.NB, PS = S / 2;          // stages come in pairs: one barrier phase
   const uint32_t XB = (uint32_t)NB * 128;
   uint8_t* xs = smem;                                            // S x XB (1024-aligned)
   uint8_t* ps = xs + (size_t)S * XB;                             // kPStages x kPBytes
-  uint64_t* full = reinterpret_cast<uint64_t*>(ps + kPStages * kPBytes);
-  uint64_t* empty = full + kMaxStages;
-  uint64_t* pfull = empty + kMaxStages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ps + kPStages * kPBytes);   // per stage pair
+  uint64_t* empty = full + kMaxStages / 2;
+  uint64_t* pfull = empty + kMaxStages / 2;
   uint64_t* pempty = pfull + kPStages;
   uint64_t* accf = pempty + kPStages;
   uint64_t* recvf = accf + 1;                                    // split-K slices received
@@ -118,11 +118,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   const int b0 = (int)((int64_t)p.B * split / p.splits);
   const int nblk = (int)((int64_t)p.B * (split + 1) / p.splits) - b0;
   const int nks = nblk * kStepsPerBlock;
+  const int npairs = nks / 2;
 
   ptx::griddep_launch_dependents();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(&full[s], kDecWarps + 1);     // 8 decoder warps + the X producer (with tx)
+    for (int s = 0; s < PS; ++s) {
+      ptx::mbar_init(&full[s], kDecWarps + 2);     // 8 decoder warps + both X producers (with tx)
       ptx::mbar_init(&empty[s], 1);                // MMA commit
     }
     for (int s = 0; s < kPStages; ++s) {
@@ -155,17 +156,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     uint64_t pol_x;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_x));
     ptx::griddep_wait();           // X may be the previous kernel's output
-    int s = warp >> 1, round = 0;
-    for (int i = warp >> 1; i < nks; i += 2) {
-      if (round > 0 && !ptx::mbar_wait(&empty[s], (uint32_t)((round - 1) & 1), limit)) {
+    const int u = warp >> 1;      // this producer loads the even (0) or odd (1) step of each pair
+    int pr = 0, round = 0;
+    for (int k = 0; k < npairs; ++k) {
+      if (round > 0 && !ptx::mbar_wait(&empty[pr], (uint32_t)((round - 1) & 1), limit)) {
         atomicExch(p.error, 21u);
         limit = 1;
       }
-      ptx::mbar_arrive_expect_tx(&full[s], XB);
-      ptx::tma_load_2d(xs + (size_t)s * XB, &xmap, (b0 * kStepsPerBlock + i) * BK, m_tile * NB,
-                       &full[s], pol_x);
-      s += 2;
-      if (s >= S) { s -= S; ++round; }
+      ptx::mbar_arrive_expect_tx(&full[pr], XB);
+      ptx::tma_load_2d(xs + (size_t)(2 * pr + u) * XB, &xmap, (b0 * kStepsPerBlock + 2 * k + u) * BK,
+                       m_tile * NB, &full[pr], pol_x);
+      if (++pr == PS) { pr = 0; ++round; }
     }
   } else if (warp == 3 && lane == 0) {
     // -------------------------------------------------- packed weight producer
@@ -188,22 +189,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
                            | ((uint32_t)(NB >> 3) << 17)     // N
                            | ((uint32_t)(kRows >> 4) << 24); // M = 128; A, B: f16, K-major
     const uint32_t xs_u = ptx::smem_u32(xs);
-    int s = 0;
+    int pr = 0;
     uint32_t ph = 0;
-    for (int i = 0; i < nks; ++i) {
-      if (!ptx::mbar_wait(&full[s], ph, limit)) {
+    for (int k = 0; k < npairs; ++k) {
+      if (!ptx::mbar_wait(&full[pr], ph, limit)) {
         atomicExch(p.error, 23u);
         limit = 1;
       }
       ptx::tc_fence_after();
-      const uint64_t bdesc = ptx::sw128_kmajor_desc(xs_u + (uint32_t)s * XB);
-      const uint32_t a_tm = tmem + (uint32_t)(kAColBase + s * kACols);
 #pragma unroll
-      for (int k = 0; k < BK / 16; ++k)
-        ptx::umma_f16_ts(tmem, a_tm + (uint32_t)(8 * k), bdesc + (uint64_t)(2 * k), idesc,
-                         (i > 0 || k > 0) ? 1u : 0u);
-      ptx::umma_commit(&empty[s]);
-      if (++s == S) { s = 0; ph ^= 1u; }
+      for (int u = 0; u < 2; ++u) {
+        const int s = 2 * pr + u;
+        const uint64_t bdesc = ptx::sw128_kmajor_desc(xs_u + (uint32_t)s * XB);
+        const uint32_t a_tm = tmem + (uint32_t)(kAColBase + s * kACols);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          ptx::umma_f16_ts(tmem, a_tm + (uint32_t)(8 * kk), bdesc + (uint64_t)(2 * kk), idesc,
+                           (k > 0 || u > 0 || kk > 0) ? 1u : 0u);
+      }
+      ptx::umma_commit(&empty[pr]);
+      if (++pr == PS) { pr = 0; ph ^= 1u; }
     }
     ptx::umma_commit(accf);
   } else if (warp >= kFirstDec) {
@@ -215,7 +220,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     const uint32_t row_off = (uint32_t)(r * 64 + 8 * h);
     const uint32_t swz = (uint32_t)((r >> 1) & 3);
     __half dnext = nvalid ? __ldg(drow) : __float2half(0.f);
-    int s = 0, round = 0, pst = 0;
+    int pr = 0, round = 0, pst = 0;
     uint32_t pph = 0;
     for (int j = 0; j < nblk; ++j) {
       const __half2 dd = __halves2half2(dnext, dnext);
@@ -232,28 +237,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       if (lane == 0) ptx::mbar_arrive(&pempty[pst]);
       if (++pst == kPStages) { pst = 0; pph ^= 1u; }
 #pragma unroll
-      for (int t = 0; t < kStepsPerBlock; ++t) {
-        if (round > 0 && !ptx::mbar_wait(&empty[s], (uint32_t)((round - 1) & 1), limit)) {
+      for (int t2 = 0; t2 < kStepsPerBlock / 2; ++t2) {
+        if (round > 0 && !ptx::mbar_wait(&empty[pr], (uint32_t)((round - 1) & 1), limit)) {
           atomicExch(p.error, 25u);
           limit = 1;
         }
         ptx::tc_fence_after();
         __syncwarp();                    // tcgen05.st below is warp-collective
-        uint32_t a[16];
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          const uint32_t w = b < 4 ? wv[t].x : wv[t].y;
-          const uint32_t sel = (uint32_t)(b & 3) * 0x0101u + 0x4040u;   // byte b into both halves
-          const uint32_t spread = __byte_perm(w, 0u, sel);
-          a[2 * b] = pair_of<0>(spread, dd);
-          a[2 * b + 1] = pair_of<1>(spread, dd);
+        for (int u = 0; u < 2; ++u) {
+          const uint2 w2 = wv[2 * t2 + u];
+          uint32_t a[16];
+#pragma unroll
+          for (int b = 0; b < 8; ++b) {
+            const uint32_t w = b < 4 ? w2.x : w2.y;
+            const uint32_t sel = (uint32_t)(b & 3) * 0x0101u + 0x4040u;   // byte b into both halves
+            const uint32_t spread = __byte_perm(w, 0u, sel);
+            a[2 * b] = pair_of<0>(spread, dd);
+            a[2 * b + 1] = pair_of<1>(spread, dd);
+          }
+          ptx::tmem_st_32x32b_x16(lane_base + (uint32_t)(kAColBase + (2 * pr + u) * kACols + 16 * h), a);
         }
-        ptx::tmem_st_32x32b_x16(lane_base + (uint32_t)(kAColBase + s * kACols + 16 * h), a);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&full[s]);
-        if (++s == S) { s = 0; ++round; }
+        if (lane == 0) ptx::mbar_arrive(&full[pr]);
+        if (++pr == PS) { pr = 0; ++round; }
       }
     }
     if (!ptx::mbar_wait(accf, 0, limit)) atomicExch(p.error, 26u);
