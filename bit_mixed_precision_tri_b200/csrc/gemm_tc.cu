@@ -23,13 +23,15 @@
 //    ring of A slots in tensor memory with tcgen05.st, so the decoded weights
 //    never touch shared memory and X needs no reordering;
 //  * one thread issues tcgen05.mma (M = 128, N = NB, K = 16, fp32 accumulate)
-//    with A in tensor memory and the activations in shared memory; a stage's
-//    commit frees both its activation buffer and its A slot;
+//    with A in tensor memory and the activations in shared memory.  That
+//    thread is a serial latency chain, so stages move in pairs: one barrier
+//    wait, eight MMAs and one commit per 128 of K; the commit frees both
+//    activation buffers and both A slots of the pair;
 //  * the epilogue reads the accumulator with tcgen05.ld.  When K is split, the
-//    CTAs of the cluster send each other 32-column slices of their partial
-//    sums through distributed shared memory; each slice's owner adds the
-//    partials in cluster-rank order, so results are deterministic.  No global
-//    scratch and no inter-CTA tickets are involved.
+//    CTAs of the cluster each own some 32-column slices of the tile: the
+//    others write their partial slices to an L2-resident scratch, the cluster
+//    synchronises once, and each owner adds the slices in cluster-rank order,
+//    so results are deterministic (no atomics, no tickets).
 #include <cudaTypedefs.h>
 
 #include "sm100_ptx.cuh"
@@ -51,16 +53,17 @@ constexpr int kDecWarps = 8;
 constexpr int kThreads = (kFirstDec + kDecWarps) * 32;
 constexpr int kRingBudget = 192 * 1024;
 constexpr int kMinSmem = 120 * 1024;              // > half an SM: one CTA (and TMEM owner) per SM
-constexpr int kRecvStride = 36;                   // floats per staged row slice (32 + pad)
-constexpr int kChunkBytes = kRows * kRecvStride * 4;  // one 32-column slice of a partial tile
+constexpr int kChunkF4 = kRows * 8;               // one 32-column slice of a partial tile (float4)
 
 // most chunks a rank sends (it owns at least floor(nch / sp) of the nch chunks)
 __host__ __device__ constexpr int max_out_chunks(int nch, int sp) { return nch - nch / sp; }
-__host__ __device__ constexpr int max_own_chunks(int nch, int sp) { return (nch + sp - 1) / sp; }
+// chunks below c that rank `rank` owns
+__host__ __device__ constexpr int owned_below(int c, int rank, int sp) { return c > rank ? (c - rank + sp - 1) / sp : 0; }
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 struct TcParams {
   unsigned* error;
+  float4* scratch;     // split-K partial slices [tile][rank][out chunk][8][128] (float4)
   int M, N, K, B;      // B = K / 256 blocks
   int NB;              // activation rows per tile (MMA N)
   int S;               // activation stages (even, <= kMaxStages)
@@ -69,7 +72,7 @@ struct TcParams {
 
 size_t smem_bytes(int NB, int S) {
   const size_t need = 1024 + (size_t)S * NB * 128 + (size_t)kPStages * kPBytes +
-                      (kMaxStages + 2 * kPStages + 2) * 8 + 16;
+                      (kMaxStages + 2 * kPStages + 1) * 8 + 16;
   return need < (size_t)kMinSmem ? (size_t)kMinSmem : need;
 }
 
@@ -110,8 +113,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   uint64_t* pfull = empty + kMaxStages / 2;
   uint64_t* pempty = pfull + kPStages;
   uint64_t* accf = pempty + kPStages;
-  uint64_t* recvf = accf + 1;                                    // split-K slices received
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recvf + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
@@ -131,7 +133,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       ptx::mbar_init(&pempty[s], kDecWarps);
     }
     ptx::mbar_init(accf, 1);
-    ptx::mbar_init(recvf, 1);
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -276,44 +277,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   const int mtile0 = m_tile * NB;
   if (p.splits > 1) {
     // Split K: chunk c of the accumulator belongs to rank c % sp.  Each CTA
-    // stages the chunks it does not own in its (now idle) rings, then one
-    // thread bulk-copies each to its owner; owners add the slices in rank order.
+    // writes the chunks it does not own to an L2-resident scratch (a warp
+    // store covers 512 contiguous bytes), the cluster synchronises once, and
+    // each owner adds the slices in rank order.
     const int sp = p.splits;
-    const uint32_t area = ptx::smem_u32(xs);
-    const int nown = split < nch ? (nch - 1 - split) / sp + 1 : 0;
-    const uint32_t recv0 = (uint32_t)(max_out_chunks(nch, sp) * kChunkBytes);
+    const int mo = max_out_chunks(nch, sp);
+    const size_t tile = (size_t)m_tile * gridDim.x + n_tile;
     if (dec) {
+      float4* mine = p.scratch + (tile * sp + split) * mo * kChunkF4 + r;
       for (int c = h; c < nch; c += 2) {
         if (c % sp == split) continue;
         uint32_t v[32];
         ptx::tmem_ld_32x32b_x32(lane_base + (uint32_t)(32 * c), v);
         ptx::tmem_ld_wait();
-        const int before = c > split ? (c - split + sp - 1) / sp : 0;    // owned chunks below c
-        const uint32_t row = area + (uint32_t)((c - before) * kChunkBytes + r * kRecvStride * 4);
+        float4* dst = mine + (size_t)(c - owned_below(c, split, sp)) * kChunkF4;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) ptx::sts128u(row + 16u * g, v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-      }
-      ptx::fence_proxy_async();
-    }
-    if (threadIdx.x == 0)
-      ptx::mbar_arrive_expect_tx(recvf, (uint32_t)(nown * (sp - 1) * kChunkBytes));
-    ptx::cluster_sync();               // staged slices written; every receive area is idle
-    if (threadIdx.x == 0) {
-      int o = 0;
-      for (int c = 0; c < nch; ++c) {
-        const int owner = c % sp;
-        if (owner == split) continue;
-        const int slot = (c / sp) * (sp - 1) + (split < owner ? split : split - 1);
-        ptx::bulk_s2peer(ptx::mapa(area + recv0 + (uint32_t)(slot * kChunkBytes), (uint32_t)owner),
-                         area + (uint32_t)(o * kChunkBytes), (uint32_t)kChunkBytes,
-                         ptx::mapa(ptx::smem_u32(recvf), (uint32_t)owner));
-        ++o;
+        for (int g = 0; g < 8; ++g)
+          dst[g * kRows] = make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                                       __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
       }
     }
-    if (dec && !ptx::mbar_wait(recvf, 0, limit)) atomicExch(p.error, 27u);
-    ptx::cluster_sync();               // every slice landed: sources may be released
+    ptx::cluster_sync();               // release / acquire at cluster scope orders the slices
     __syncwarp();
     if (dec) {                         // warp-uniform: tcgen05.ld is warp-collective
+      const int nown = split < nch ? (nch - 1 - split) / sp + 1 : 0;
       for (int lc = h; lc < nown; lc += 2) {
         const int c = lc * sp + split;
         uint32_t v[32];
@@ -328,15 +315,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
             for (int e = 0; e < 32; ++e) acc[e] += __uint_as_float(v[e]);
             continue;
           }
-          const int slot = lc * (sp - 1) + (src < split ? src : src - 1);
-          const uint32_t a = area + recv0 + (uint32_t)(slot * kChunkBytes + r * kRecvStride * 4);
+          const float4* srcp = p.scratch + ((tile * sp + src) * mo + (c - owned_below(c, src, sp))) * kChunkF4 + r;
 #pragma unroll
           for (int g = 0; g < 8; ++g) {
-            const uint4 f = ptx::lds128(a + 16u * g);
-            acc[4 * g] += __uint_as_float(f.x);
-            acc[4 * g + 1] += __uint_as_float(f.y);
-            acc[4 * g + 2] += __uint_as_float(f.z);
-            acc[4 * g + 3] += __uint_as_float(f.w);
+            const float4 f = __ldcg(srcp + g * kRows);
+            acc[4 * g] += f.x;
+            acc[4 * g + 1] += f.y;
+            acc[4 * g + 2] += f.z;
+            acc[4 * g + 3] += f.w;
           }
         }
 #pragma unroll
@@ -365,7 +351,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 // ---------------------------------------------------------------- host side
 struct Plan {
   int NB, S, tiles_n, tiles_m, splits;
-  size_t smem;
+  size_t smem, scratch;
 };
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -439,8 +425,6 @@ Plan plan_for(int64_t M, int64_t N, int64_t K, int num_sms) {
   pl.splits = 1;
   for (int sp = 1; sp <= 4; ++sp) {
     if (sp > B) break;
-    const int64_t area = (int64_t)(max_out_chunks(nch, sp) + max_own_chunks(nch, sp) * (sp - 1)) * kChunkBytes;
-    if (sp > 1 && area > (int64_t)pl.S * XB + (int64_t)kPStages * kPBytes) continue;
     const int64_t slots = sp == 1 ? num_sms : cluster_slots(sp, num_sms);
     const int64_t waves = ceil_div(tiles * sp, slots);
     const double t = (double)waves * ((double)ceil_div(B, sp) * kStepsPerBlock + (sp == 1 ? 6.0 : 9.0));
@@ -450,6 +434,7 @@ Plan plan_for(int64_t M, int64_t N, int64_t K, int num_sms) {
     }
   }
   pl.smem = smem_bytes(pl.NB, pl.S);
+  pl.scratch = pl.splits > 1 ? (size_t)tiles * pl.splits * max_out_chunks(nch, pl.splits) * kChunkF4 * 16 : 0;
   return pl;
 }
 
@@ -460,7 +445,10 @@ bool gemm_tc_supported(int fmt, int64_t M, int64_t N, int64_t K) {
          ceil_div(M, 256) <= 65535;
 }
 
-size_t gemm_tc_ws_bytes(int, int64_t, int64_t, int64_t, int) { return 256; }
+size_t gemm_tc_ws_bytes(int fmt, int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (!gemm_tc_supported(fmt, M, N, K)) return 256;
+  return 256 + plan_for(M, N, K, num_sms).scratch;
+}
 
 cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __half* d, __half* Y,
                            int M, int N, int K, void* ws, int num_sms, cudaStream_t s) {
@@ -491,6 +479,7 @@ cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __
   }
   TcParams p;
   p.error = static_cast<unsigned*>(ws);
+  p.scratch = reinterpret_cast<float4*>(static_cast<uint8_t*>(ws) + 256);
   p.M = M; p.N = N; p.K = K; p.B = K / kBlock;
   p.NB = pl.NB; p.S = pl.S; p.splits = pl.splits;
   if (pl.smem > (size_t)kMaxSmem) return cudaErrorInvalidValue;
