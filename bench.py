@@ -51,8 +51,8 @@ WORKLOADS = {
                          seeds=[10, 11, 12, 13, 14, 15, 16]),
 }
 # path -> launches of this library's kernels per GEMM call (prep + main for the
-# tensor-core paths; TQ1 adds its transcode)
-KERNELS_PER_CALL = {1: 1, 2: 2, 3: 2, 4: 1}
+# mma.sync path, one kernel otherwise; TQ1 adds its transcode)
+KERNELS_PER_CALL = {1: 1, 2: 2, 3: 1, 4: 1}
 
 
 def workload_from_args(name, M=None, fmt=None):

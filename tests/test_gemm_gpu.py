@@ -233,3 +233,72 @@ def test_i8_path_workspace_shared_with_other_paths():
         _check(Y1, X1, trits, d)
         Y8 = tri.gemm(torch.from_numpy(X8).to(DEV), qd, dd, N, K, "tq2", workspace=ws, path=tri.PATH_MMA)
         _check(Y8, X8, trits, d)
+
+
+@pytest.mark.parametrize("M,N,K", [(17, 384, 512), (33, 256, 1024), (300, 520, 2304), (513, 384, 1280),
+                                   (1024, 256, 768), (256, 1000, 11008), (129, 8192, 1024)])
+def test_tcgen05_path_shapes(M, N, K):
+    """The tensor-memory kernel at shapes that exercise its tiling: activation
+    tiles of 32..256 rows (ragged last tile), ragged weight tiles, several
+    activation tiles, and K split over clusters of 2..4 CTAs (few tiles, many
+    blocks) including a split whose parts hold different numbers of blocks."""
+    X, trits, qs, d = _case(M, N, K, 400 + M + N % 89, "tq2", per_block=True, p_zero=0.31)
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, "tq2", path=tri.PATH_TCGEN05)
+    _check(Y, X, trits, d)
+
+
+def test_tcgen05_path_deterministic_split_k():
+    """Split-K partial sums are added in cluster-rank order: bitwise repeatable."""
+    M, N, K = 256, 2048, 8192
+    X, trits, qs, d = _case(M, N, K, 71, "tq2")
+    args = (torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV),
+            N, K, "tq2")
+    Y1 = tri.gemm(*args, path=tri.PATH_TCGEN05)
+    Y2 = tri.gemm(*args, path=tri.PATH_TCGEN05)
+    assert torch.equal(Y1, Y2)
+    rows = np.arange(0, N, 37)
+    _check(Y1[:, rows], X, trits[rows], d[rows])
+
+
+def test_tcgen05_path_graph_replay_new_inputs():
+    """A captured call replayed with new activations in the same buffers: the
+    split-K scratch in the workspace is rewritten by every replay."""
+    M, N, K = 96, 1024, 6144
+    X, trits, qs, d = _case(M, N, K, 72, "tq2")
+    Xd = torch.from_numpy(X).to(DEV)
+    qd, dd = torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV)
+    Y = torch.empty(M, N, dtype=torch.float16, device=DEV)
+    ws = tri.Workspace(DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        tri.gemm(Xd, qd, dd, N, K, "tq2", out=Y, workspace=ws, stream=s, path=tri.PATH_TCGEN05)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        tri.gemm(Xd, qd, dd, N, K, "tq2", out=Y, workspace=ws, stream=s, path=tri.PATH_TCGEN05)
+    for seed in (17, 18):
+        Xn = inputs.activations(M, K, seed).numpy()
+        Xd.copy_(torch.from_numpy(Xn).to(DEV))
+        g.replay()
+        torch.cuda.synchronize()
+        _check(Y, Xn, trits, d)
+
+
+def test_tcgen05_path_back_to_back_layers():
+    """Consecutive launches chained by programmatic dependent launch: each
+    layer reads the previous layer's output as its activations."""
+    M, K = 64, 1024
+    trits1, g1 = O.absmean_ternarize(inputs.latent_weights(K, K, 81).numpy(), 1e-6)
+    trits2, g2 = O.absmean_ternarize(inputs.latent_weights(K, K, 82).numpy(), 1e-6)
+    q1, d1 = O.pack("tq2", trits1, np.array([g1], np.float32))
+    q2, d2 = O.pack("tq2", trits2, np.array([g2], np.float32))
+    X = inputs.activations(M, K, 83).numpy() * np.float16(0.05)
+    Xd = torch.from_numpy(X).to(DEV)
+    H = tri.gemm(Xd, torch.from_numpy(q1).to(DEV), torch.from_numpy(d1).to(DEV), K, K, "tq2",
+                 path=tri.PATH_TCGEN05)
+    Y = tri.gemm(H, torch.from_numpy(q2).to(DEV), torch.from_numpy(d2).to(DEV), K, K, "tq2",
+                 path=tri.PATH_TCGEN05)
+    Hh = H.cpu().numpy()
+    _check(H, X, trits1, d1)
+    _check(Y, Hh, trits2, d2)
