@@ -354,21 +354,38 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int m = 0; m < M; ++m) sum[h][m] = acc[h][m];
-    for (long long cc = cfirst + 1; cc <= clast; ++cc) {
-      const unsigned long long* src = p.partials + (size_t)cc * kRT * M;
+    // The partial sums of up to kBatch contributors are loaded together (one
+    // round trip), then checked and added in CTA order; only a value whose
+    // stamp is not yet this call's is polled again.
+    constexpr int kBatch = 8;
+    for (long long c0 = cfirst + 1; c0 <= clast; c0 += kBatch) {
+      const int nb = (int)(clast - c0 + 1 < kBatch ? clast - c0 + 1 : kBatch);
+      unsigned long long v[kBatch][2][M];
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+      for (int k = 0; k < kBatch; ++k)
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const unsigned long long* a = src + (r_local + 8 * h) * M + m;
-          unsigned long long v = ld_relaxed_u64(a);
-          for (int spin = 0; (v >> 32) != stamp && spin < kSpinLimit; ++spin) {
-            __nanosleep(64);
-            v = ld_relaxed_u64(a);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int m = 0; m < M; ++m)
+            v[k][h][m] = k < nb ? ld_relaxed_u64(p.partials + (size_t)(c0 + k) * kRT * M + (r_local + 8 * h) * M + m)
+                                : 0ull;
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        if (k >= nb) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int m = 0; m < M; ++m) {
+            unsigned long long x = v[k][h][m];
+            const unsigned long long* a = p.partials + (size_t)(c0 + k) * kRT * M + (r_local + 8 * h) * M + m;
+            for (int spin = 0; (x >> 32) != stamp && spin < kSpinLimit; ++spin) {
+              __nanosleep(64);
+              x = ld_relaxed_u64(a);
+            }
+            if ((x >> 32) != stamp) atomicOr(p.error, 1u);
+            sum[h][m] += __uint_as_float((unsigned)x);
           }
-          if ((v >> 32) != stamp) atomicOr(p.error, 1u);
-          sum[h][m] += __uint_as_float((unsigned)v);
-        }
+      }
     }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
