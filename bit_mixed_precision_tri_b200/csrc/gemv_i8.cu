@@ -648,7 +648,8 @@ cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half
 // Shapes whose per-CTA block pairs fit in shared memory with two CTAs per SM
 // (every CTA of the grid must be resident at once: reducers wait for others).
 bool gemv_i8_supported(int64_t M, int64_t N, int64_t K) {
-  if (M < 1 || M > 2 || N < 1 || K < kBlock || K % kBlock) return false;
+  if (M >= 3) return gemv_i8n_supported(M, N, K);
+  if (M < 1 || N < 1 || K < kBlock || K % kBlock) return false;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
   static std::once_flag once[kMaxDev];
@@ -664,6 +665,7 @@ bool gemv_i8_supported(int64_t M, int64_t N, int64_t K) {
 }
 
 size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M >= 3) return gemv_i8n_ws_bytes(M, N, K, num_sms);
   return layout_for(M, N, K, num_sms).total;
 }
 
@@ -671,7 +673,7 @@ cudaError_t launch_gemv_i8(const __half* X, const uint8_t* qs, const __half* d, 
                            int N, int K, void* ws, int num_sms, cudaStream_t s) {
   if (M == 1) return launch_m<1>(X, qs, d, Y, N, K, ws, num_sms, s);
   if (M == 2) return launch_m<2>(X, qs, d, Y, N, K, ws, num_sms, s);
-  return cudaErrorNotSupported;
+  return launch_gemv_i8n(X, qs, d, Y, M, N, K, ws, num_sms, s);
 }
 
 }  // namespace tri

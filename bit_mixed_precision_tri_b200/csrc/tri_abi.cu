@@ -84,7 +84,7 @@ size_t path_ws_bytes(int fmt, int path, int64_t M, int64_t N, int64_t K, int sms
 }
 
 int auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
-  if (M <= 2 && path_supported(fmt, TRI_PATH_I8, M, N, K)) return TRI_PATH_I8;
+  if (M <= 16 && path_supported(fmt, TRI_PATH_I8, M, N, K)) return TRI_PATH_I8;
   if (M <= 16 && path_supported(fmt, TRI_PATH_MMA, M, N, K)) return TRI_PATH_MMA;
   if (M > 16 && path_supported(fmt, TRI_PATH_TCGEN05, M, N, K)) return TRI_PATH_TCGEN05;
   return TRI_PATH_SIMT;

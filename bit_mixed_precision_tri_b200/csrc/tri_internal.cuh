@@ -49,7 +49,12 @@ cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const _
                             __half* Y, int M, int N, int K, void* ws, int num_sms,
                             cudaStream_t s);
 
-// decode-regime integer tensor-core path (TQ2, M <= 2)
+// decode-regime integer tensor-core path (TQ2, M <= 16: gemv_i8.cu for M <= 2,
+// gemv_i8n.cu for 3 <= M <= 16)
+bool gemv_i8n_supported(int64_t M, int64_t N, int64_t K);
+size_t gemv_i8n_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv_i8n(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M, int N,
+                            int K, void* ws, int num_sms, cudaStream_t s);
 bool gemv_i8_supported(int64_t M, int64_t N, int64_t K);
 size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemv_i8(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M,

@@ -83,8 +83,8 @@ typedef enum tri_gemm_path {
     TRI_PATH_SIMT = 1,     /* CUDA-core kernel, any M (correctness baseline)           */
     TRI_PATH_MMA = 2,      /* decode-regime tensor-core kernel, M <= 16                */
     TRI_PATH_TCGEN05 = 3,  /* compute-regime kernel: tcgen05 MMA, TMEM accumulators    */
-    TRI_PATH_I8 = 4        /* decode-regime int8 tensor-core kernel (exact integer
-                              products with 24-bit fixed-point X), M <= 2            */
+    TRI_PATH_I8 = 4        /* decode-regime int8 tensor-core kernels (exact integer
+                              products with 24-bit fixed-point X), M <= 16           */
 } tri_gemm_path;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -185,8 +185,9 @@ TRI_API tri_status tri_unpack(int format, const uint8_t* qs, int64_t N, int64_t 
  *             N, K) bytes, 256-byte aligned; its contents on entry do not
  *             matter (each call initialises what it uses).  Calls that share
  *             one workspace must be ordered (same stream, or events).
- *   path      TRI_PATH_AUTO chooses TRI_PATH_I8 for M <= 2, TRI_PATH_MMA
- *             for M <= 16 and TRI_PATH_TCGEN05 above (TQ1 weights are first
+ *   path      TRI_PATH_AUTO chooses TRI_PATH_I8 for M <= 16 (TRI_PATH_MMA
+ *             where it cannot serve the shape) and TRI_PATH_TCGEN05 above
+ *             (TQ1 weights are first
  *             transcoded to TQ2 in the workspace on those three paths); an
  *             explicit path that cannot serve the shape returns
  *             TRI_ERR_NOT_IMPLEMENTED.  TRI_PATH_I8 quantises each

@@ -302,3 +302,63 @@ def test_tcgen05_path_back_to_back_layers():
     Hh = H.cpu().numpy()
     _check(H, X, trits1, d1)
     _check(Y, Hh, trits2, d2)
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+@pytest.mark.parametrize("M,N,K", [(3, 384, 512), (5, 1000, 2304), (9, 129, 256), (12, 2048, 4096),
+                                   (16, 520, 11008), (16, 4096, 28672), (8, 1024, 8192)])
+def test_i8_path_batch_up_to_16(fmt, M, N, K):
+    """The integer path for 3 <= M <= 16 (three or six column tiles of digits):
+    ragged row tiles, K split over clusters of 1..8 CTAs, per-block scales."""
+    X, trits, qs, d = _case(M, N, K, 500 + M + N % 83, fmt, per_block=True, p_zero=0.31)
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, fmt, path=tri.PATH_I8)
+    rows = np.arange(N) if N <= 2048 else np.arange(0, N, 41)
+    _check(Y[:, rows], X, trits[rows], d[rows])
+
+
+@pytest.mark.parametrize("M", [4, 16])
+def test_i8_path_batch_activation_extremes(M):
+    """Per (block, batch row) quantisation steps: rows with different ranges, a
+    huge value among tiny ones, zero blocks and signed extremes."""
+    N, K = 384, 2048
+    X, trits, qs, d = _case(M, N, K, 42, "tq2", per_block=True, p_zero=0.5)
+    X = X.copy()
+    X[0, 0] = 60000.0
+    X[0, 1:256] = (np.random.default_rng(4).standard_normal(255) * 1e-3).astype(np.float16)
+    X[1 % M, 256:512] = 0.0
+    X[M - 1, 512:768] = np.float16(6e-8)
+    X[:, 768] = -65504.0
+    X[:, 769] = 65504.0
+    X[M // 2] *= np.float16(1e-3)
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, "tq2", path=tri.PATH_I8)
+    _check(Y, X, trits, d)
+
+
+def test_i8_path_batch_deterministic_and_graph_replay():
+    """Split-K sums in cluster-rank order are bitwise repeatable, and a captured
+    call replayed with new activations recomputes its activation records."""
+    M, N, K = 16, 2048, 8192
+    X, trits, qs, d = _case(M, N, K, 73, "tq2")
+    Xd = torch.from_numpy(X).to(DEV)
+    qd, dd = torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV)
+    Y1 = tri.gemm(Xd, qd, dd, N, K, "tq2", path=tri.PATH_I8)
+    Y2 = tri.gemm(Xd, qd, dd, N, K, "tq2", path=tri.PATH_I8)
+    assert torch.equal(Y1, Y2)
+    Y = torch.empty(M, N, dtype=torch.float16, device=DEV)
+    ws = tri.Workspace(DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        tri.gemm(Xd, qd, dd, N, K, "tq2", out=Y, workspace=ws, stream=s, path=tri.PATH_I8)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        tri.gemm(Xd, qd, dd, N, K, "tq2", out=Y, workspace=ws, stream=s, path=tri.PATH_I8)
+    for seed in (27, 28):
+        Xn = inputs.activations(M, K, seed).numpy()
+        Xd.copy_(torch.from_numpy(Xn).to(DEV))
+        g.replay()
+        torch.cuda.synchronize()
+        rows = np.arange(0, N, 13)
+        _check(Y[:, rows], Xn, trits[rows], d[rows])
