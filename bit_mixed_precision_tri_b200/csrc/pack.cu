@@ -175,13 +175,15 @@ unpack_tq1_kernel(const uint8_t* __restrict__ qs, int64_t N, int64_t K, int8_t* 
 }
 
 // TQ1 -> TQ2 transcode, so the tensor-core GEMM paths can consume TQ1
-// weights: one warp per (row, block) turns 52 TQ1 bytes into sixteen TQ2
+// weights: one thread per (row, block) turns 52 TQ1 bytes into sixteen TQ2
 // words.  A per-CTA table maps each byte value to its five digits as 2-bit
-// fields (first weight lowest), built with the multiply-by-3 decoder.
+// fields (first weight lowest), built with the multiply-by-3 decoder; the
+// fields of consecutive bytes form one 512-bit stream (10 bits per byte, 2
+// for the last byte's single weight), cut into 32-bit words at compile-time
+// offsets.
 __global__ void __launch_bounds__(kThreads)
 transcode_tq1_tq2_kernel(const uint8_t* __restrict__ qs1, int64_t rowblocks, uint32_t* __restrict__ qs2) {
   __shared__ uint16_t lut[256];
-  __shared__ uint32_t words[kThreads / 32][16];
   for (int i = threadIdx.x; i < 256; i += kThreads) {
     unsigned v = (unsigned)i, code = 0u;
 #pragma unroll
@@ -193,26 +195,32 @@ transcode_tq1_tq2_kernel(const uint8_t* __restrict__ qs1, int64_t rowblocks, uin
     lut[i] = (uint16_t)code;
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t stride = (int64_t)gridDim.x * (kThreads / 32);
-  for (int64_t rb = (int64_t)blockIdx.x * (kThreads / 32) + warp; rb < rowblocks; rb += stride) {
-    if (lane < 16) words[warp][lane] = 0u;
-    __syncwarp();
-    if (lane < 26) {
-      const uint8_t* src = qs1 + rb * kTq1BlockBytes + 2 * lane;
-      const unsigned c0 = lut[src[0]];
-      unsigned c1 = lut[src[1]];
-      if (lane == 25) c1 &= 3u;                    // byte 51 holds one weight
-      const unsigned v = c0 | (c1 << 10);          // 20 bits at bit 20 * lane
-      const int bit = 20 * lane, w = bit >> 5, sh = bit & 31;
-      atomicOr(&words[warp][w], v << sh);
-      // the 20-bit field spills into the next word; lane 25's field (bits
-      // 500..511 in use) ends inside word 15, so there is no word 16 to touch
-      if (sh > 12 && w + 1 < 16) atomicOr(&words[warp][w + 1], v >> (32 - sh));
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t rb = (int64_t)blockIdx.x * kThreads + threadIdx.x; rb < rowblocks; rb += stride) {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(qs1 + rb * kTq1BlockBytes);
+    uint32_t in[kTq1BlockBytes / 4];
+#pragma unroll
+    for (int j = 0; j < kTq1BlockBytes / 4; ++j) in[j] = __ldg(src + j);
+    uint32_t out[16];
+    uint64_t acc = 0;
+    int nbits = 0, o = 0;
+#pragma unroll
+    for (int i = 0; i < kTq1BlockBytes; ++i) {
+      const unsigned byte = (in[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+      unsigned code = lut[byte];
+      const int nb = i == kTq1BlockBytes - 1 ? 2 : 10;   // byte 51 holds one weight
+      if (nb == 2) code &= 3u;
+      acc |= (uint64_t)code << nbits;
+      nbits += nb;
+      if (nbits >= 32) {
+        out[o++] = (uint32_t)acc;
+        acc >>= 32;
+        nbits -= 32;
+      }
     }
-    __syncwarp();
-    if (lane < 16) qs2[rb * 16 + lane] = words[warp][lane];
-    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(qs2 + rb * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
   }
 }
 
@@ -221,7 +229,7 @@ transcode_tq1_tq2_kernel(const uint8_t* __restrict__ qs1, int64_t rowblocks, uin
 cudaError_t launch_transcode_tq1_tq2(const uint8_t* qs1, int64_t N, int64_t K, uint8_t* qs2,
                                      cudaStream_t s) {
   const int64_t rowblocks = N * (K / kBlock);
-  int64_t g = ceil_div(rowblocks, kThreads / 32);
+  int64_t g = ceil_div(rowblocks, kThreads);
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
