@@ -99,12 +99,13 @@ __device__ __forceinline__ void store_y(__half* __restrict__ Y, const uint32_t (
     if (e < lim) Y[(size_t)(mbase + e) * N + n] = __float2half_rn(__uint_as_float(v[e]));
 }
 
+template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap qmap,
                const __half* __restrict__ dsc, __half* __restrict__ Y, const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.S, NB = p.NB, PS = S / 2;          // stages come in pairs: one barrier phase
+  const int S = p.S, NB = p.NB, PS = S / G;          // stages move in groups of G: one barrier phase
   const uint32_t XB = (uint32_t)NB * 128;
   uint8_t* xs = smem;                                            // S x XB (1024-aligned)
   uint8_t* ps = xs + (size_t)S * XB;                             // kPStages x kPBytes
@@ -120,7 +121,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
   const int b0 = (int)((int64_t)p.B * split / p.splits);
   const int nblk = (int)((int64_t)p.B * (split + 1) / p.splits) - b0;
   const int nks = nblk * kStepsPerBlock;
-  const int npairs = nks / 2;
+  const int ngroups = nks / G;
 
   ptx::griddep_launch_dependents();
   if (threadIdx.x == 0) {
@@ -157,16 +158,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     uint64_t pol_x;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol_x));
     ptx::griddep_wait();           // X may be the previous kernel's output
-    const int u = warp >> 1;      // this producer loads the even (0) or odd (1) step of each pair
+    const int u = warp >> 1;      // this producer loads the even (0) or odd (1) steps of each group
     int pr = 0, round = 0;
-    for (int k = 0; k < npairs; ++k) {
+    for (int k = 0; k < ngroups; ++k) {
       if (round > 0 && !ptx::mbar_wait(&empty[pr], (uint32_t)((round - 1) & 1), limit)) {
         atomicExch(p.error, 21u);
         limit = 1;
       }
-      ptx::mbar_arrive_expect_tx(&full[pr], XB);
-      ptx::tma_load_2d(xs + (size_t)(2 * pr + u) * XB, &xmap, (b0 * kStepsPerBlock + 2 * k + u) * BK,
-                       m_tile * NB, &full[pr], pol_x);
+      ptx::mbar_arrive_expect_tx(&full[pr], XB * (G / 2));
+#pragma unroll
+      for (int v = u; v < G; v += 2)
+        ptx::tma_load_2d(xs + (size_t)(G * pr + v) * XB, &xmap, (b0 * kStepsPerBlock + G * k + v) * BK,
+                         m_tile * NB, &full[pr], pol_x);
       if (++pr == PS) { pr = 0; ++round; }
     }
   } else if (warp == 3 && lane == 0) {
@@ -192,15 +195,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     const uint32_t xs_u = ptx::smem_u32(xs);
     int pr = 0;
     uint32_t ph = 0;
-    for (int k = 0; k < npairs; ++k) {
+    for (int k = 0; k < ngroups; ++k) {
       if (!ptx::mbar_wait(&full[pr], ph, limit)) {
         atomicExch(p.error, 23u);
         limit = 1;
       }
       ptx::tc_fence_after();
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int s = 2 * pr + u;
+      for (int u = 0; u < G; ++u) {
+        const int s = G * pr + u;
         const uint64_t bdesc = ptx::sw128_kmajor_desc(xs_u + (uint32_t)s * XB);
         const uint32_t a_tm = tmem + (uint32_t)(kAColBase + s * kACols);
 #pragma unroll
@@ -238,7 +241,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       if (lane == 0) ptx::mbar_arrive(&pempty[pst]);
       if (++pst == kPStages) { pst = 0; pph ^= 1u; }
 #pragma unroll
-      for (int t2 = 0; t2 < kStepsPerBlock / 2; ++t2) {
+      for (int t2 = 0; t2 < kStepsPerBlock / G; ++t2) {
         if (round > 0 && !ptx::mbar_wait(&empty[pr], (uint32_t)((round - 1) & 1), limit)) {
           atomicExch(p.error, 25u);
           limit = 1;
@@ -246,8 +249,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         ptx::tc_fence_after();
         __syncwarp();                    // tcgen05.st below is warp-collective
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint2 w2 = wv[2 * t2 + u];
+        for (int u = 0; u < G; ++u) {
+          const uint2 w2 = wv[G * t2 + u];
           uint32_t a[16];
 #pragma unroll
           for (int b = 0; b < 8; ++b) {
@@ -257,7 +260,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
             a[2 * b] = pair_of<0>(spread, dd);
             a[2 * b + 1] = pair_of<1>(spread, dd);
           }
-          ptx::tmem_st_32x32b_x16(lane_base + (uint32_t)(kAColBase + (2 * pr + u) * kACols + 16 * h), a);
+          ptx::tmem_st_32x32b_x16(lane_base + (uint32_t)(kAColBase + (G * pr + u) * kACols + 16 * h), a);
         }
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
@@ -375,7 +378,9 @@ cudaError_t ensure_smem_attr() {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 16 && done[dev]) return cudaSuccess;
-  e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  e = cudaFuncSetAttribute(gemm_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemm_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSmem);
   if (e == cudaSuccess && dev >= 0 && dev < 16) done[dev] = true;
   return e;
 }
@@ -400,7 +405,7 @@ int cluster_slots(int sp, int num_sms) {
     attr[0].val.clusterDim.z = (unsigned)sp;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel, &cfg) != cudaSuccess) clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<2>, &cfg) != cudaSuccess) clusters = 0;
   }
   cudaGetLastError();
   slot = clusters > 0 ? clusters * sp : (num_sms / sp) * sp;
@@ -499,7 +504,10 @@ cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __
   attr[1].val.clusterDim.z = (unsigned)pl.splits;
   cfg.attrs = attr;
   cfg.numAttrs = pl.splits > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel, xmap, qmap, d, Y, p);
+  // small activation tiles make each MMA short: move K in groups of four
+  // steps per barrier phase to amortise the issuing thread's waits
+  if (pl.NB <= 128 && pl.S % 4 == 0) return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<4>, xmap, qmap, d, Y, p);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<2>, xmap, qmap, d, Y, p);
 }
 
 }  // namespace tri
