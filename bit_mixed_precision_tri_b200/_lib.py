@@ -45,6 +45,8 @@ SIGNATURES = {
     "tri_gemm_tq2": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p]),
     "tri_gemm_tq1": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p]),
     "tri_gemm_auto_path": (_i, [_i, _i64, _i64, _i64]),
+    "tri_gemm_swiglu_workspace_bytes": (_sz, [_i, _i64, _i64, _i64]),
+    "tri_gemm_swiglu": (_i, [_i, _i, _p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p]),
     "tri_gemm_tq2_noalloc": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p]),
     "tri_gemm_tq2_noalloc_fits": (_i, [_i64, _i64, _i64]),
 }

@@ -168,6 +168,53 @@ def gemm(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, N: int, K: int, fmt
     return Y
 
 
+def interleave_gate_up(qs_gate: torch.Tensor, d_gate: torch.Tensor, qs_up: torch.Tensor,
+                       d_up: torch.Tensor):
+    """Packed weights of a gate and an up projection (F rows each, F % 8 == 0)
+    as the 2F-row matrix that ``gemm_swiglu`` takes: rows interleaved in
+    groups of eight (fused row 16j + i = gate row 8j + i, 16j + 8 + i = up row
+    8j + i).  A one-time weight layout step (memory movement only)."""
+    F = qs_gate.shape[0]
+    if F % 8 or qs_up.shape != qs_gate.shape or d_up.shape != d_gate.shape:
+        raise ValueError("gate and up must have the same shape, with a multiple of 8 rows")
+
+    def inter(a, b):
+        a = a.reshape(F // 8, 8, -1)
+        b = b.reshape(F // 8, 8, -1)
+        return torch.cat([a, b], dim=1).reshape(2 * F, -1).contiguous()
+
+    return inter(qs_gate, qs_up), inter(d_gate, d_up)
+
+
+def gemm_swiglu(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, F: int, K: int, fmt="tq2",
+                path: int = PATH_AUTO, out: torch.Tensor = None, workspace: Workspace = None,
+                stream=None) -> torch.Tensor:
+    """Y = silu(X Wg^T) * (X Wu^T), fp16 [M][F], from the interleaved 2F-row
+    packed weights of ``interleave_gate_up``."""
+    if not (X.is_cuda and qs.is_cuda and d.is_cuda):
+        raise ValueError("tensors must live on a CUDA device")
+    if not (X.is_contiguous() and qs.is_contiguous() and d.is_contiguous()):
+        raise ValueError("tensors must be contiguous")
+    if X.dtype != torch.float16:
+        raise ValueError("X must be float16")
+    M = X.shape[0]
+    f = FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+    if out is None:
+        Y = torch.empty(M, F, dtype=torch.float16, device=X.device)
+    else:
+        if not (out.is_cuda and out.is_contiguous()):
+            raise ValueError("out must be a contiguous CUDA tensor")
+        Y = out
+    L = _lib.lib()
+    ws = (workspace or _workspace_for(X.device)).get(max(int(L.tri_gemm_swiglu_workspace_bytes(f, M, F, K)), 256))
+    s = stream.cuda_stream if stream is not None else _stream(X.device)
+    st = L.tri_gemm_swiglu(f, int(path), X.data_ptr(), qs.data_ptr(), d.data_ptr(), Y.data_ptr(),
+                           M, F, K, ws.data_ptr(), ws.numel(), s)
+    if st:
+        _lib.check(st, "tri_gemm_swiglu")
+    return Y
+
+
 class TernaryLinear:
     """A ternary linear layer: absmean-ternarized, packed weights and a GEMM.
 

@@ -31,6 +31,11 @@
 //  * Split K.  A 128-row tile's blocks may be split over the CTAs of a
 //    thread-block cluster; partial sums go through an L2-resident scratch and
 //    rank 0 adds them in rank order after one cluster barrier: deterministic.
+//  * SwiGLU epilogue (optional).  With gate and up rows interleaved in groups
+//    of eight, the two rows a thread holds (r and r + 8) are the gate and up
+//    projections of one output feature, and it writes silu(g) * u directly
+//    (the feed-forward unit of "Scaling Laws and Efficient Inference for
+//    Ternary Language Models", section "The model").
 #include <cudaTypedefs.h>
 
 #include "sm100_ptx.cuh"
@@ -59,6 +64,7 @@ struct NParams {
   float* scratch;          // [tile][rank][128][M]
   unsigned* error;
   int M, N, K, B, splits, stages;
+  int swiglu;              // N = 2F fused gate/up rows, Y = silu(gate) * up, [M][F]
 };
 
 // ---------------------------------------------------------------- prep kernel
@@ -135,6 +141,9 @@ i8n_prep_kernel(const __half* __restrict__ X, int M, int K, uint8_t* __restrict_
     sc[16 + m] = (float)sum;                   // sum_k x^_k
   }
 }
+
+// silu(g) * u in fp32 (silu(g) = g / (1 + e^-g))
+__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + expf(-g)) * u; }
 
 // ---------------------------------------------------------------- main kernel
 template <int NT>
@@ -271,12 +280,17 @@ i8n_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restrict__ 
 
   // ---------------------------------------------------------------- epilogue
   const int M = p.M;
+  const int F = p.N / 2;
   if (p.splits == 1) {
     if (warp < kConsumers) {
 #pragma unroll
       for (int k = 0; k < T; ++k) {
         const int m = T * tig + k;
-        if (m < M) {
+        if (m >= M) continue;
+        if (p.swiglu) {
+          const int f = tile * (kRows / 2) + warp * 8 + gid;    // rows n0 (gate), n1 = n0 + 8 (up)
+          if (n0 < p.N) Y[(size_t)m * F + f] = __float2half_rn(silu_mul(y[k][0], y[k][1]));
+        } else {
           if (n0 < p.N) Y[(size_t)m * p.N + n0] = __float2half_rn(y[k][0]);
           if (n1 < p.N) Y[(size_t)m * p.N + n1] = __float2half_rn(y[k][1]);
         }
@@ -297,11 +311,23 @@ i8n_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restrict__ 
     ptx::cluster_sync();
     if (split == 0) {
       const float* base = p.scratch + (size_t)tile * p.splits * kRows * M;
-      for (int i = threadIdx.x; i < kRows * M; i += kThreads) {
-        const int r = i / M, m = i % M, n = tile * kRows + r;
-        float v = 0.f;
-        for (int sp = 0; sp < p.splits; ++sp) v += __ldcg(base + (size_t)sp * kRows * M + i);
-        if (n < p.N) Y[(size_t)m * p.N + n] = __float2half_rn(v);
+      if (p.swiglu) {
+        for (int i = threadIdx.x; i < (kRows / 2) * M; i += kThreads) {
+          const int q = i / M, m = i % M, rg = 16 * (q >> 3) + (q & 7), f = tile * (kRows / 2) + q;
+          float g = 0.f, u = 0.f;
+          for (int sp = 0; sp < p.splits; ++sp) {
+            g += __ldcg(base + (size_t)sp * kRows * M + rg * M + m);
+            u += __ldcg(base + (size_t)sp * kRows * M + (rg + 8) * M + m);
+          }
+          if (tile * kRows + rg < p.N) Y[(size_t)m * F + f] = __float2half_rn(silu_mul(g, u));
+        }
+      } else {
+        for (int i = threadIdx.x; i < kRows * M; i += kThreads) {
+          const int r = i / M, m = i % M, n = tile * kRows + r;
+          float v = 0.f;
+          for (int sp = 0; sp < p.splits; ++sp) v += __ldcg(base + (size_t)sp * kRows * M + i);
+          if (n < p.N) Y[(size_t)m * p.N + n] = __float2half_rn(v);
+        }
       }
     }
   }
@@ -364,7 +390,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn_n() {
 
 template <int NT>
 cudaError_t launch_nt(const NPlan& pl, const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M,
-                      int N, int K, void* ws, cudaStream_t s) {
+                      int N, int K, void* ws, bool swiglu, cudaStream_t s) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   auto enc = encode_fn_n();
   if (!enc) return cudaErrorNotSupported;
@@ -407,6 +433,7 @@ cudaError_t launch_nt(const NPlan& pl, const __half* X, const uint8_t* qs, const
   p.scratch = reinterpret_cast<float*>(w + pl.off_scr);
   p.error = reinterpret_cast<unsigned*>(w);
   p.M = M; p.N = N; p.K = K; p.B = B; p.splits = pl.splits; p.stages = pl.S;
+  p.swiglu = swiglu ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)pl.tiles, 1, (unsigned)pl.splits);
   cfg.blockDim = dim3(kThreads);
@@ -435,11 +462,12 @@ size_t gemv_i8n_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
 }
 
 cudaError_t launch_gemv_i8n(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M, int N, int K,
-                            void* ws, int num_sms, cudaStream_t s) {
+                            void* ws, int num_sms, cudaStream_t s, bool swiglu) {
   if (!gemv_i8n_supported(M, N, K)) return cudaErrorNotSupported;
+  if (swiglu && N % 16 != 0) return cudaErrorNotSupported;
   const NPlan pl = nplan(M, N, K, num_sms);
-  if (pl.NT == 3) return launch_nt<3>(pl, X, qs, d, Y, M, N, K, ws, s);
-  return launch_nt<6>(pl, X, qs, d, Y, M, N, K, ws, s);
+  if (pl.NT == 3) return launch_nt<3>(pl, X, qs, d, Y, M, N, K, ws, swiglu, s);
+  return launch_nt<6>(pl, X, qs, d, Y, M, N, K, ws, swiglu, s);
 }
 
 }  // namespace tri

@@ -252,6 +252,78 @@ tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs, 
   }
 }
 
+namespace {
+// the fused epilogue serves 3 <= M <= 16 on the integer path
+bool swiglu_fused(int path, int64_t M) { return path == TRI_PATH_I8 && M >= 3 && M <= 16; }
+}  // namespace
+
+size_t tri_gemm_swiglu_workspace_bytes(int format, int64_t M, int64_t F, int64_t K) {
+  if (F < 8 || F % 8 != 0) return 0;
+  const size_t g = tri_gemm_workspace_bytes(format, M, 2 * F, K);
+  if (g == 0) return 0;
+  return up256(g) + up256((size_t)M * 2 * F * 2);
+}
+
+tri_status tri_gemm_swiglu(int format, int path, const uint16_t* X, const uint8_t* qs, const uint16_t* d,
+                           uint16_t* Y, int64_t M, int64_t F, int64_t K, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (format != TRI_TQ2 && format != TRI_TQ1) return TRI_ERR_INVALID_ARG;
+  if (path < TRI_PATH_AUTO || path > TRI_PATH_I8) return TRI_ERR_INVALID_ARG;
+  if (!X || !qs || !d || !Y) return TRI_ERR_INVALID_ARG;
+  if (M < 1 || M > kMaxDim) return TRI_ERR_SHAPE;
+  if (F < 8 || F % 8 != 0 || F > kMaxDim / 2) return TRI_ERR_SHAPE;
+  const int64_t N = 2 * F;
+  tri_status st = check_nk(N, K);
+  if (st != TRI_OK) return st;
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(d, 4)) return TRI_ERR_ALIGNMENT;
+  if (!aligned(qs, format == TRI_TQ2 ? 16 : 4)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  if ((st = device_info(&di)) != TRI_OK) return st;
+  if (path == TRI_PATH_AUTO) path = auto_path(format, M, N, K);
+  if (!path_supported(format, path, M, N, K)) return TRI_ERR_NOT_IMPLEMENTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __half* Xh = reinterpret_cast<const __half*>(X);
+  const __half* dh = reinterpret_cast<const __half*>(d);
+  __half* Yh = reinterpret_cast<__half*>(Y);
+  const size_t gemm_need = path == TRI_PATH_SIMT ? 0 : path_ws_bytes(format, path, M, N, K, di.sms);
+  const bool fused = swiglu_fused(path, M);
+  const size_t need = fused ? gemm_need : up256(gemm_need) + up256((size_t)M * N * 2);
+  if (need && (!workspace || workspace_bytes < need)) return TRI_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
+  const uint8_t* q2 = qs;
+  uint8_t* inner = static_cast<uint8_t*>(workspace);
+  if (format == TRI_TQ1 && path != TRI_PATH_SIMT) {
+    uint8_t* t = static_cast<uint8_t*>(workspace);
+    const cudaError_t e = tri::launch_transcode_tq1_tq2(qs, N, K, t, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    q2 = t;
+    inner = t + transcode_bytes(format, path, N, K);
+  }
+  if (fused)
+    return from_cuda(tri::launch_gemv_i8n(Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner, di.sms, s, true));
+  // unfused: the [M][2F] product into the workspace tail, then the combine
+  __half* G2 = reinterpret_cast<__half*>(static_cast<uint8_t*>(workspace) + up256(gemm_need));
+  cudaError_t e = cudaSuccess;
+  switch (path) {
+    case TRI_PATH_SIMT:
+      e = tri::launch_gemm_simt(format, Xh, qs, dh, G2, (int)M, (int)N, (int)K, s);
+      break;
+    case TRI_PATH_MMA:
+      e = tri::launch_gemv_mma(TRI_TQ2, Xh, q2, dh, G2, (int)M, (int)N, (int)K, inner, di.sms, s);
+      break;
+    case TRI_PATH_I8:
+      e = tri::launch_gemv_i8(Xh, q2, dh, G2, (int)M, (int)N, (int)K, inner, di.sms, s);
+      break;
+    case TRI_PATH_TCGEN05:
+      e = tri::launch_gemm_tc(TRI_TQ2, Xh, q2, dh, G2, (int)M, (int)N, (int)K, inner, di.sms, s);
+      break;
+    default:
+      return TRI_ERR_INVALID_ARG;
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  return from_cuda(tri::launch_swiglu_combine(G2, Yh, M, F, s));
+}
+
 int tri_gemm_tq2_noalloc_fits(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || M > 16 || check_nk(N, K) != TRI_OK) return 0;
   DevInfo di;

@@ -53,8 +53,11 @@ cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const _
 // gemv_i8n.cu for 3 <= M <= 16)
 bool gemv_i8n_supported(int64_t M, int64_t N, int64_t K);
 size_t gemv_i8n_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+// swiglu: N = 2F rows of gate and up interleaved in groups of 8, Y = silu(gate) * up [M][F]
 cudaError_t launch_gemv_i8n(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M, int N,
-                            int K, void* ws, int num_sms, cudaStream_t s);
+                            int K, void* ws, int num_sms, cudaStream_t s, bool swiglu = false);
+// silu(G) * U from a [M][2F] fp16 product in the interleaved row order, into Y [M][F]
+cudaError_t launch_swiglu_combine(const __half* G2, __half* Y, int64_t M, int64_t F, cudaStream_t s);
 bool gemv_i8_supported(int64_t M, int64_t N, int64_t K);
 size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemv_i8(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M,

@@ -229,6 +229,30 @@ TRI_API tri_status tri_gemm_tq2_noalloc(const uint16_t* X, const uint8_t* qs, co
 /* 1 if tri_gemm_tq2_noalloc accepts this shape on the current device, else 0. */
 TRI_API int tri_gemm_tq2_noalloc_fits(int64_t M, int64_t N, int64_t K);
 
+/* ------------------------------------------------------------------------
+ * Fused gate/up projection with a SwiGLU epilogue: the gated feed-forward
+ * unit of "Scaling Laws and Efficient Inference for Ternary Language
+ * Models" (section "The model"; its MLP is a SwiGLU over two ternary
+ * projections):
+ *   Y[m][f] = silu(G[m][f]) * U[m][f],  silu(g) = g / (1 + e^-g),
+ *   G = X (d_g W_hat_g)^T, U = X (d_u W_hat_u)^T, fp32 accumulation, fp16 Y.
+ *   qs, d     the 2F rows of both packed weight matrices (format as in
+ *             tri_gemm), interleaved in groups of eight rows: fused row
+ *             16j + i is gate row 8j + i and fused row 16j + 8 + i is up row
+ *             8j + i (i < 8).  F % 8 == 0.
+ *   Y         device fp16[M][F], 16-byte aligned, written.
+ *   workspace at least tri_gemm_swiglu_workspace_bytes(format, M, F, K).
+ *   path      as in tri_gemm for the 2F-row product.  For 3 <= M <= 16 the
+ *             integer kernel applies silu(g) * u to the fp32 sums in its
+ *             epilogue; other paths write the [M][2F] product (fp16) into
+ *             the workspace and a second kernel combines it.
+ *   Errors as tri_gemm; F % 8 != 0 returns TRI_ERR_SHAPE.
+ * ---------------------------------------------------------------------- */
+TRI_API size_t tri_gemm_swiglu_workspace_bytes(int format, int64_t M, int64_t F, int64_t K);
+TRI_API tri_status tri_gemm_swiglu(int format, int path, const uint16_t* X, const uint8_t* qs,
+                                   const uint16_t* d, uint16_t* Y, int64_t M, int64_t F, int64_t K,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* Kernel that tri_gemm would launch for this call under TRI_PATH_AUTO
  * (one of tri_gemm_path), or -1 if the shape is invalid. */
 TRI_API int tri_gemm_auto_path(int format, int64_t M, int64_t N, int64_t K);

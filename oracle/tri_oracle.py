@@ -286,6 +286,43 @@ def gemm_tolerance(X, d, y_ref, rows=None) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# a7 (next row): gated feed-forward unit  [TLS "The model": the MLP is a
+# SwiGLU over two ternary projections]
+# --------------------------------------------------------------------------
+def silu_f64(g) -> np.ndarray:
+    """silu(g) = g / (1 + e^-g) = g * sigmoid(g), float64, stable for large |g|."""
+    g = np.asarray(g, dtype=np.float64)
+    e = np.exp(-np.abs(g))
+    sig = np.where(g >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return g * sig
+
+
+def swiglu_f64(X, trits_gate, d_gate, trits_up, d_up):
+    """Y[m][f] = silu(G[m][f]) * U[m][f] with G, U the two ternary products
+    (gemm_f64, not rounded).  Returns (Y, G, U)."""
+    G = gemm_f64(X, trits_gate, d_gate)
+    U = gemm_f64(X, trits_up, d_up)
+    return silu_f64(G) * U, G, U
+
+
+def swiglu_tolerance(X, d_gate, d_up, G, U) -> np.ndarray:
+    """Allowed |y - y_ref| for the fused SwiGLU output.
+
+    Each product may be off by its GEMM tolerance T (gemm_tolerance) and, on
+    paths that store it, by fp16 rounding of the product (2^-11 relative);
+    silu has slope at most 1.0999 (attained near g = 2.4), so
+    |silu(g') u' - silu(g) u| <= 1.1 T_g (|u| + T_u) + |silu(g)| T_u, plus
+    2^-10 |y| for the fp32 arithmetic and the fp16 rounding of y.
+    """
+    Tg = gemm_tolerance(X, d_gate, G)
+    Tu = gemm_tolerance(X, d_up, U)
+    Tg = Tg + 2.0 ** -11 * (np.abs(G) + Tg)
+    Tu = Tu + 2.0 ** -11 * (np.abs(U) + Tu)
+    Y = silu_f64(G) * U
+    return 1.1 * Tg * (np.abs(U) + Tu) + np.abs(silu_f64(G)) * Tu + 2.0 ** -10 * np.abs(Y)
+
+
+# --------------------------------------------------------------------------
 # size identities  [TLS "2 bits per weight", "1.6 bits per weight",
 # "Fast inference on CPUs"]
 # --------------------------------------------------------------------------

@@ -362,3 +362,44 @@ def test_i8_path_batch_deterministic_and_graph_replay():
         torch.cuda.synchronize()
         rows = np.arange(0, N, 13)
         _check(Y[:, rows], Xn, trits[rows], d[rows])
+
+
+def _swiglu_case(M, F, K, seed, fmt, per_block=True):
+    rng = np.random.default_rng(seed)
+    tg = inputs.random_trits(F, K, 0.31, seed).numpy()
+    tu = inputs.random_trits(F, K, 0.31, seed + 1).numpy()
+    sg = inputs.block_scales(F, K, seed + 2).numpy() if per_block else np.array([0.03], np.float32)
+    su = inputs.block_scales(F, K, seed + 3).numpy() if per_block else np.array([0.02], np.float32)
+    qg, dg = O.pack(fmt, tg, sg)
+    qu, du = O.pack(fmt, tu, su)
+    X = inputs.activations(M, K, seed + 4).numpy()
+    q, d = tri.interleave_gate_up(torch.from_numpy(qg), torch.from_numpy(dg), torch.from_numpy(qu),
+                                  torch.from_numpy(du))
+    return X, tg, dg, tu, du, q.to(DEV), d.to(DEV)
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+@pytest.mark.parametrize("M,F,K", [(1, 520, 2304), (2, 128, 512), (4, 520, 2304), (16, 1024, 8192),
+                                   (9, 64, 256), (40, 264, 1024), (16, 8, 256)])
+def test_gemm_swiglu_vs_oracle(fmt, M, F, K):
+    """silu(X Wg^T) * (X Wu^T) on every regime: fused epilogue (3 <= M <= 16,
+    split K included) and the product-then-combine route (M <= 2, M > 16)."""
+    X, tg, dg, tu, du, q, d = _swiglu_case(M, F, K, 600 + M + F % 37, fmt)
+    Y = tri.gemm_swiglu(torch.from_numpy(X).to(DEV), q, d, F, K, fmt)
+    y = Y.float().cpu().numpy().astype(np.float64)
+    ref, G, U = O.swiglu_f64(X, tg, dg, tu, du)
+    tol = O.swiglu_tolerance(X, dg, du, G, U)
+    bad = np.abs(y - ref) > tol
+    assert not bad.any(), f"{bad.sum()} outputs out of tolerance; worst {(np.abs(y - ref) - tol).max()}"
+
+
+def test_gemm_swiglu_fused_matches_separate_products():
+    """The fused epilogue agrees with two plain GEMMs combined on the host."""
+    M, F, K = 16, 2048, 4096
+    X, tg, dg, tu, du, q, d = _swiglu_case(M, F, K, 77, "tq2", per_block=False)
+    Xd = torch.from_numpy(X).to(DEV)
+    Y = tri.gemm_swiglu(Xd, q, d, F, K, "tq2", path=tri.PATH_I8).float()
+    Y2 = tri.gemm(Xd, q, d, 2 * F, K, "tq2", path=tri.PATH_I8).float().reshape(M, F // 8, 2, 8)
+    g, u = Y2[:, :, 0, :].reshape(M, F), Y2[:, :, 1, :].reshape(M, F)
+    ref = torch.nn.functional.silu(g) * u
+    assert torch.allclose(Y, ref, rtol=2e-3, atol=2e-3)

@@ -362,3 +362,53 @@ def test_pins_catch_planted_mistakes():
     x = np.array(g["W"], np.float32)
     away = (np.sign(x) * np.floor(np.abs(np.clip(x, -1, 1)) + 0.5)).astype(np.int8)
     assert away.tolist() != g["trits_half_to_even"]
+
+
+# ---------------------------------------------------------------- a7 SwiGLU
+def test_silu_closed_forms():
+    """silu(g) = g / (1 + e^-g): values fixed by the definition."""
+    g = np.array([0.0, 1.0, -1.0, 2.0, 30.0, -40.0, -745.0])
+    want = np.array([0.0, 1 / (1 + math.exp(-1)), -1 / (1 + math.exp(1)), 2 / (1 + math.exp(-2)),
+                     30.0 / (1 + math.exp(-30)), -40.0 * math.exp(-40) / (1 + math.exp(-40)), -0.0])
+    got = O.silu_f64(g)
+    assert np.allclose(got, want, rtol=1e-15, atol=1e-300)
+    assert abs(O.silu_f64(1.0) - 0.7310585786300049) < 1e-15     # sigmoid(1)
+    assert np.all(np.isfinite(O.silu_f64(np.array([1e308, -1e308]))))
+
+
+def test_swiglu_hand_example():
+    """One row, one block: gate trits pick +x_0 - x_1, up trits sum x_0..x_3,
+    so Y = silu(d_g (x0 - x1)) * d_u (x0 + x1 + x2 + x3)."""
+    K = 256
+    X = np.zeros((1, K), np.float16)
+    X[0, :4] = [1.5, -0.5, 0.25, 2.0]
+    tg = np.zeros((1, K), np.int8)
+    tg[0, 0], tg[0, 1] = 1, -1
+    tu = np.zeros((1, K), np.int8)
+    tu[0, :4] = 1
+    dg = np.array([[0.5]], np.float16)
+    du = np.array([[0.25]], np.float16)
+    Y, G, U = O.swiglu_f64(X, tg, dg, tu, du)
+    g = 0.5 * (1.5 + 0.5)
+    u = 0.25 * (1.5 - 0.5 + 0.25 + 2.0)
+    assert G[0, 0] == g and U[0, 0] == u
+    assert abs(Y[0, 0] - g / (1 + math.exp(-g)) * u) < 1e-15
+
+
+def test_swiglu_zero_gate_and_tolerance_bounds():
+    """An all-zero gate gives Y = 0 exactly; the tolerance is positive, and a
+    planted error of 2x the tolerance in the gate product is rejected."""
+    rng = np.random.default_rng(5)
+    X = rng.standard_normal((3, 512)).astype(np.float16)
+    tu = rng.integers(-1, 2, (16, 512)).astype(np.int8)
+    du = np.full((16, 2), 0.03, np.float16)
+    tg = np.zeros((16, 512), np.int8)
+    Y, G, U = O.swiglu_f64(X, tg, du, tu, du)
+    assert np.all(Y == 0.0)
+    tg = rng.integers(-1, 2, (16, 512)).astype(np.int8)
+    Y, G, U = O.swiglu_f64(X, tg, du, tu, du)
+    tol = O.swiglu_tolerance(X, du, du, G, U)
+    assert np.all(tol > 0)
+    Tg = O.gemm_tolerance(X, du, G)
+    bad = O.silu_f64(G + 4 * Tg + 1e-3) * U
+    assert np.any(np.abs(bad - Y) > tol)
