@@ -49,10 +49,22 @@ WORKLOADS = {
     "block70b_m16": dict(layers=[(8192, 8192), (1024, 8192), (1024, 8192), (8192, 8192),
                                  (28672, 8192), (28672, 8192), (8192, 28672)], M=16, fmt="tq2",
                          seeds=[10, 11, 12, 13, 14, 15, 16]),
+    # the same block with q/k/v concatenated into one GEMM and gate/up fused
+    # with the SwiGLU epilogue (2 x 28672 interleaved rows -> 28672 outputs)
+    "block70b_m16_fused": dict(layers=[(10240, 8192), (8192, 8192), (57344, 8192), (8192, 28672)],
+                               M=16, fmt="tq2", seeds=[10, 13, 14, 16], swiglu=[2]),
 }
-# path -> launches of this library's kernels per GEMM call (prep + main for the
-# mma.sync path, one kernel otherwise; TQ1 adds its transcode)
-KERNELS_PER_CALL = {1: 1, 2: 2, 3: 1, 4: 1}
+def kernels_per_call(path, M, fmt, swiglu=False):
+    """Launches of this library's kernels for one call: prep + main for the
+    mma.sync path and for the integer path at 3 <= M <= 16, one kernel
+    otherwise; TQ1 adds its transcode on the tensor-core paths; an unfused
+    SwiGLU call adds its combine kernel."""
+    n = 2 if path == 2 or (path == 4 and M >= 3) else 1
+    if fmt == "tq1" and path != 1:
+        n += 1
+    if swiglu and not (path == 4 and 3 <= M <= 16):
+        n += 1
+    return n
 
 
 def workload_from_args(name, M=None, fmt=None):
@@ -172,8 +184,9 @@ def prepare_layers(w, device, copies):
         del trits
         reps = [(qs, d)] + [(qs.clone(), d.clone()) for _ in range(copies - 1)]
         X = inputs.activations(w["M"], K, 6 + w["M"] + seed).to(device)
-        Y = torch.empty(w["M"], N, dtype=torch.float16, device=device)
-        layers.append(dict(N=N, K=K, reps=reps, X=X, Y=Y, gamma=float(g.item())))
+        sw = len(layers) in w.get("swiglu", ())
+        Y = torch.empty(w["M"], N // 2 if sw else N, dtype=torch.float16, device=device)
+        layers.append(dict(N=N, K=K, reps=reps, X=X, Y=Y, gamma=float(g.item()), swiglu=sw))
     torch.cuda.synchronize(device)
     return layers
 
@@ -184,19 +197,29 @@ def run_ours(args, rank, world, device, w=None):
         w = workload_from_args(args.workload, args.M, args.fmt)
     M, fmt = w["M"], w["fmt"]
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    step_bytes = sum(algo_bytes(fmt, M, N, K) for N, K in w["layers"])
+    step_bytes = sum(algo_bytes(fmt, M, N, K) - (M * N if i in w.get("swiglu", ()) else 0)
+                     for i, (N, K) in enumerate(w["layers"]))
     weight_bytes = sum(N * tri.packed_row_bytes(fmt, K) + N * (K // 256) * 2 for N, K in w["layers"])
     copies = max(args.steps, int(np.ceil(3 * l2 / max(weight_bytes, 1))) + 1)
     layers = prepare_layers(w, device, copies)
     paths = [tri.auto_path(fmt, M, L["N"], L["K"]) for L in layers]
     ws = tri.Workspace(device)
-    ws.get(max(tri.gemm_workspace_bytes(fmt, M, L["N"], L["K"]) for L in layers))
+    from bit_mixed_precision_tri_b200 import _lib as _tl
+    ws.get(max(max(tri.gemm_workspace_bytes(fmt, M, L["N"], L["K"]),
+                   int(_tl.lib().tri_gemm_swiglu_workspace_bytes(tri.api.FORMATS[fmt], M, L["N"] // 2, L["K"]))
+                   if L["swiglu"] else 0) for L in layers))
     stream = torch.cuda.Stream(device)
+
+    def call(L, X, qs, d, Y):
+        if L["swiglu"]:
+            tri.gemm_swiglu(X, qs, d, L["N"] // 2, L["K"], fmt, out=Y, workspace=ws, stream=stream)
+        else:
+            tri.gemm(X, qs, d, L["N"], L["K"], fmt, out=Y, workspace=ws, stream=stream)
 
     def step(c):
         for L in layers:
             qs, d = L["reps"][c]
-            tri.gemm(L["X"], qs, d, L["N"], L["K"], fmt, out=L["Y"], workspace=ws, stream=stream)
+            call(L, L["X"], qs, d, L["Y"])
 
     # eager warm-up (also allocates), then the warm-up and the timed steps are
     # each captured as one CUDA graph (one launch for the whole region; the
@@ -237,14 +260,15 @@ def run_ours(args, rank, world, device, w=None):
     # back on one stream: the average launch takes elapsed / launches
     n_launch = args.steps * len(layers)
     kernel_ms = elapsed_ms
-    kernel_bytes = args.steps * sum(algo_bytes(fmt, M, L["N"], L["K"]) for L in layers)
+    kernel_bytes = args.steps * sum(algo_bytes(fmt, M, L["N"], L["K"]) - (M * L["N"] if L["swiglu"] else 0)
+                                    for L in layers)
     max_ms = allreduce_max(elapsed_ms, world, device)
 
     # end-to-end through the public API: every step copies its inputs (the X
     # of every layer, one pinned host buffer) to the device, runs the GEMMs
     # with eager calls, and reads all outputs back (one pinned host buffer)
     xsz = [M * L["K"] for L in layers]
-    ysz = [M * L["N"] for L in layers]
+    ysz = [L["Y"].numel() for L in layers]
     xh = torch.cat([L["X"].flatten().cpu() for L in layers]).pin_memory()
     yh = torch.empty(sum(ysz), dtype=torch.float16).pin_memory()
     xd_all = torch.empty(sum(xsz), dtype=torch.float16, device=device)
@@ -252,7 +276,7 @@ def run_ours(args, rank, world, device, w=None):
     xd = list(torch.split(xd_all, xsz))
     yd = list(torch.split(yd_all, ysz))
     xd = [x.view(M, L["K"]) for x, L in zip(xd, layers)]
-    yd = [y.view(M, L["N"]) for y, L in zip(yd, layers)]
+    yd = [y.view(M, -1) for y, L in zip(yd, layers)]
     h2d, d2h = xh.numel() * 2, yh.numel() * 2
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -266,16 +290,14 @@ def run_ours(args, rank, world, device, w=None):
                 xd_all.copy_(xh, non_blocking=True)
                 for i, L in enumerate(layers):
                     qs, d = L["reps"][c]
-                    tri.gemm(xd[i], qs, d, L["N"], L["K"], fmt, out=yd[i], workspace=ws,
-                             stream=stream)
+                    call(L, xd[i], qs, d, yd[i])
                 yh.copy_(yd_all, non_blocking=True)
             if rep == 1:
                 e1.record(stream)
             torch.cuda.synchronize(device)
     e2e_ms = allreduce_max(e0.elapsed_time(e1), world, device)
     del g_warm, g_steps
-    launches = args.steps * sum(KERNELS_PER_CALL.get(p, 1) + (1 if fmt == "tq1" and p != 1 else 0)
-                                for p in paths)
+    launches = args.steps * sum(kernels_per_call(p, M, fmt, L["swiglu"]) for p, L in zip(paths, layers))
     unit = "GB/s" if M <= 32 else "TFLOP/s"
     flops = sum(2.0 * M * N * K for N, K in w["layers"])
 
@@ -521,6 +543,7 @@ def run_sweep(args, rank, world, device):
         for M in SWEEP_M:
             jobs.append(dict(name=f"sweep_8192_{fmt}_m{M}", layers=[(8192, 8192)], M=M, fmt=fmt, seeds=[5]))
     jobs.append(dict(WORKLOADS["block70b_m16"], name="block70b_m16"))
+    jobs.append(dict(WORKLOADS["block70b_m16_fused"], name="block70b_m16_fused"))
     for fmt in ("tq2", "tq1"):
         for p0 in (0.3, 0.5, 0.7, 0.9):
             for M in (1, 16, 128):
