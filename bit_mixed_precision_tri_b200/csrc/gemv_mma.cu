@@ -32,7 +32,6 @@
 //  * Partial sums of a row tile split across CTAs are combined by the last
 //    CTA to finish (an atomic ticket, no waiting), in CTA order, so results
 //    are deterministic.
-#include <cstdlib>
 #include <mutex>
 
 #include <cudaTypedefs.h>
@@ -524,26 +523,17 @@ cudaError_t launch_mp(const __half* X, const uint8_t* qs, const __half* d, __hal
 
 }  // namespace
 
-// The decode-regime path runs the mma.sync kernel above; the tcgen05 kernel
-// (gemv_tc.cu) is selectable for comparison (TRI_DECODE_KERNEL=tc).
-bool use_legacy_decode() {
-  const char* e = std::getenv("TRI_DECODE_KERNEL");
-  return !(e && e[0] == 't');
-}
-
 bool gemv_mma_supported(int fmt, int64_t M, int64_t N, int64_t K) {
   return fmt == TRI_TQ2 && M >= 1 && M <= 16 && N >= 1 && K >= kBlock && K % kBlock == 0;
 }
 
 size_t gemv_mma_ws_bytes(int, int64_t M, int64_t N, int64_t K, int num_sms) {
-  const size_t a = layout_for(M, N, K, num_sms).total, b = gemv_tc_ws_bytes(N, K, num_sms);
-  return a > b ? a : b;
+  return layout_for(M, N, K, num_sms).total;
 }
 
 cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const __half* d, __half* Y,
                             int M, int N, int K, void* ws, int num_sms, cudaStream_t s) {
   if (!gemv_mma_supported(fmt, M, N, K)) return cudaErrorNotSupported;
-  if (!use_legacy_decode()) return launch_gemv_tc(X, qs, d, Y, M, N, K, ws, num_sms, s);
   if (M <= 8) return launch_mp<8>(X, qs, d, Y, M, N, K, ws, num_sms, s);
   return launch_mp<16>(X, qs, d, Y, M, N, K, ws, num_sms, s);
 }

@@ -63,11 +63,6 @@ size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemv_i8(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M,
                            int N, int K, void* ws, int num_sms, cudaStream_t s);
 
-// decode-regime kernel on tcgen05 with decoded weights in tensor memory (TQ2, M <= 16)
-size_t gemv_tc_ws_bytes(int64_t N, int64_t K, int num_sms);
-cudaError_t launch_gemv_tc(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M, int N,
-                           int K, void* ws, int num_sms, cudaStream_t s);
-
 // decode-regime path with library-owned static scratch (no allocation)
 size_t gemv_noalloc_scratch_limit();
 size_t gemv_noalloc_scratch_need(int64_t M, int64_t N, int64_t K, int num_sms);
