@@ -175,15 +175,25 @@ unpack_tq1_kernel(const uint8_t* __restrict__ qs, int64_t N, int64_t K, int8_t* 
 }
 
 // TQ1 -> TQ2 transcode, so the tensor-core GEMM paths can consume TQ1
-// weights: one thread per (row, block) turns 52 TQ1 bytes into sixteen TQ2
-// words.  A per-CTA table maps each byte value to its five digits as 2-bit
-// fields (first weight lowest), built with the multiply-by-3 decoder; the
-// fields of consecutive bytes form one 512-bit stream (10 bits per byte, 2
-// for the last byte's single weight), cut into 32-bit words at compile-time
-// offsets.
+// weights.  A warp takes 32 consecutive (row, block) units: it copies their
+// 32 x 52 contiguous bytes into shared memory with 16-byte loads, each lane
+// turns one unit's 52 bytes into sixteen TQ2 words (a per-CTA table maps
+// each byte value to its five digits as 2-bit fields, first weight lowest,
+// built with the multiply-by-3 decoder; the fields of consecutive bytes form
+// one 512-bit stream, 10 bits per byte and 2 for the last byte's single
+// weight, cut into 32-bit words at compile-time offsets), and the warp
+// writes the 32 x 64 output bytes back with 16-byte stores.  A lane's 13
+// input words sit at a 13-word stride (odd: no bank conflicts) and its 16
+// output words at a 17-word stride.
+constexpr int kTcWarps = kThreads / 32;
+constexpr int kInWords = kTq1BlockBytes / 4;     // 13
+constexpr int kOutStride = 17;
+
 __global__ void __launch_bounds__(kThreads)
 transcode_tq1_tq2_kernel(const uint8_t* __restrict__ qs1, int64_t rowblocks, uint32_t* __restrict__ qs2) {
   __shared__ uint16_t lut[256];
+  __shared__ __align__(16) uint32_t sin[kTcWarps][32 * kInWords];
+  __shared__ uint32_t sout[kTcWarps][32 * kOutStride];
   for (int i = threadIdx.x; i < 256; i += kThreads) {
     unsigned v = (unsigned)i, code = 0u;
 #pragma unroll
@@ -195,32 +205,51 @@ transcode_tq1_tq2_kernel(const uint8_t* __restrict__ qs1, int64_t rowblocks, uin
     lut[i] = (uint16_t)code;
   }
   __syncthreads();
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t rb = (int64_t)blockIdx.x * kThreads + threadIdx.x; rb < rowblocks; rb += stride) {
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(qs1 + rb * kTq1BlockBytes);
-    uint32_t in[kTq1BlockBytes / 4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* wi = sin[warp];
+  uint32_t* wo = sout[warp];
+  const int64_t step = (int64_t)gridDim.x * kTcWarps * 32;
+  const bool a16 = (reinterpret_cast<uintptr_t>(qs1) & 15u) == 0;   // TQ1 planes need only 4-byte alignment
+  for (int64_t rb0 = ((int64_t)blockIdx.x * kTcWarps + warp) * 32; rb0 < rowblocks; rb0 += step) {
+    const int nb = rowblocks - rb0 < 32 ? (int)(rowblocks - rb0) : 32;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(qs1 + rb0 * kTq1BlockBytes);
+    const int nw = nb * kInWords;
+    if (nb == 32 && a16) {             // 416 words = 104 aligned 16-byte pieces (rb0 * 52 % 16 == 0)
+      const uint4* s4 = reinterpret_cast<const uint4*>(src);
+      for (int i = lane; i < 32 * kInWords / 4; i += 32) reinterpret_cast<uint4*>(wi)[i] = __ldg(s4 + i);
+    } else {
+      for (int i = lane; i < nw; i += 32) wi[i] = __ldg(src + i);
+    }
+    __syncwarp();
+    if (lane < nb) {
+      uint32_t in[kInWords];
 #pragma unroll
-    for (int j = 0; j < kTq1BlockBytes / 4; ++j) in[j] = __ldg(src + j);
-    uint32_t out[16];
-    uint64_t acc = 0;
-    int nbits = 0, o = 0;
+      for (int j = 0; j < kInWords; ++j) in[j] = wi[lane * kInWords + j];
+      uint64_t acc = 0;
+      int nbits = 0, o = 0;
 #pragma unroll
-    for (int i = 0; i < kTq1BlockBytes; ++i) {
-      const unsigned byte = (in[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-      unsigned code = lut[byte];
-      const int nb = i == kTq1BlockBytes - 1 ? 2 : 10;   // byte 51 holds one weight
-      if (nb == 2) code &= 3u;
-      acc |= (uint64_t)code << nbits;
-      nbits += nb;
-      if (nbits >= 32) {
-        out[o++] = (uint32_t)acc;
-        acc >>= 32;
-        nbits -= 32;
+      for (int i = 0; i < kTq1BlockBytes; ++i) {
+        const unsigned byte = (in[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+        unsigned code = lut[byte];
+        const int nbt = i == kTq1BlockBytes - 1 ? 2 : 10;   // byte 51 holds one weight
+        if (nbt == 2) code &= 3u;
+        acc |= (uint64_t)code << nbits;
+        nbits += nbt;
+        if (nbits >= 32) {
+          wo[lane * kOutStride + o++] = (uint32_t)acc;
+          acc >>= 32;
+          nbits -= 32;
+        }
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(qs2 + rb * 16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_uint4(out[4 * q], out[4 * q + 1], out[4 * q + 2], out[4 * q + 3]);
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(qs2 + rb0 * 16);
+    for (int i = lane; i < nb * 4; i += 32) {            // output word 4i .. 4i+3 of the group
+      const int u = i >> 2, o = (i & 3) * 4;
+      const uint32_t* w = wo + u * kOutStride + o;
+      dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __syncwarp();
   }
 }
 
@@ -229,7 +258,7 @@ transcode_tq1_tq2_kernel(const uint8_t* __restrict__ qs1, int64_t rowblocks, uin
 cudaError_t launch_transcode_tq1_tq2(const uint8_t* qs1, int64_t N, int64_t K, uint8_t* qs2,
                                      cudaStream_t s) {
   const int64_t rowblocks = N * (K / kBlock);
-  int64_t g = ceil_div(rowblocks, kThreads);
+  int64_t g = ceil_div(rowblocks, kThreads);      // one (row, block) unit per thread
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
