@@ -22,6 +22,7 @@ STATUS_NAMES = {
     0: "TRI_OK", 1: "TRI_ERR_INVALID_ARG", 2: "TRI_ERR_SHAPE", 3: "TRI_ERR_ALIGNMENT",
     4: "TRI_ERR_NONFINITE", 5: "TRI_ERR_INVALID_CODE", 6: "TRI_ERR_CUDA",
     7: "TRI_ERR_NOT_IMPLEMENTED", 8: "TRI_ERR_WORKSPACE", 9: "TRI_ERR_NO_DEVICE",
+    10: "TRI_ERR_SCRATCH_LIMIT",
 }
 
 _p = ctypes.c_void_p
@@ -49,6 +50,8 @@ SIGNATURES = {
     "tri_gemm_swiglu": (_i, [_i, _i, _p, _p, _p, _p, _i64, _i64, _i64, _p, _sz, _p]),
     "tri_gemm_tq2_noalloc": (_i, [_p, _p, _p, _p, _i64, _i64, _i64, _p]),
     "tri_gemm_tq2_noalloc_fits": (_i, [_i64, _i64, _i64]),
+    "tri_wait_status": (_i, [_p, _i, _p]),
+    "tri_selftest_wait_timeout": (_i, [_i, _p, _p]),
 }
 
 

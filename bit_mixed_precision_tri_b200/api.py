@@ -6,6 +6,8 @@ non-OK status and never fall back to another implementation.
 """
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from . import _lib
@@ -213,6 +215,31 @@ def gemm_swiglu(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, F: int, K: i
     if st:
         _lib.check(st, "tri_gemm_swiglu")
     return Y
+
+
+def wait_status(device=None, clear: bool = True) -> int:
+    """Synchronize the device's current stream and return its wait status
+    word: 0, or the code of the first bounded wait inside a GEMM kernel that
+    gave up since the last clear (that call's output is then unspecified)."""
+    dev = torch.device(device or "cuda")
+    code = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        st = _lib.lib().tri_wait_status(ctypes.byref(code), int(clear), _stream(dev))
+    if st:
+        _lib.check(st, "tri_wait_status")
+    return int(code.value)
+
+
+def selftest_wait_timeout(which: int, device=None) -> None:
+    """Enqueue a kernel whose bounded wait cannot complete (0: an mbarrier
+    phase, 1: a stamped word), so that it records its code (90 or 91) in the
+    wait status word; read it back with ``wait_status``."""
+    dev = torch.device(device or "cuda")
+    scratch = torch.empty(8, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.lib().tri_selftest_wait_timeout(int(which), scratch.data_ptr(), _stream(dev))
+    if st:
+        _lib.check(st, "tri_selftest_wait_timeout")
 
 
 class TernaryLinear:

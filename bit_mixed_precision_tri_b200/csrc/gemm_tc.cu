@@ -59,7 +59,7 @@ constexpr int kChunkF4 = kRows * 8;               // one 32-column slice of a pa
 __host__ __device__ constexpr int max_out_chunks(int nch, int sp) { return nch - nch / sp; }
 // chunks below c that rank `rank` owns
 __host__ __device__ constexpr int owned_below(int c, int rank, int sp) { return c > rank ? (c - rank + sp - 1) / sp : 0; }
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kWaitLimit = 1u << 18;   // mbarrier polls: ~4 us each when pending, ~1 s in all
 
 struct TcParams {
   unsigned* error;
@@ -162,7 +162,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     int pr = 0, round = 0;
     for (int k = 0; k < ngroups; ++k) {
       if (round > 0 && !ptx::mbar_wait(&empty[pr], (uint32_t)((round - 1) & 1), limit)) {
-        atomicExch(p.error, 21u);
+        ptx::record_wait_failure(p.error, 21u);
         limit = 1;
       }
       ptx::mbar_arrive_expect_tx(&full[pr], XB * (G / 2));
@@ -180,7 +180,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     uint32_t ph = 0;
     for (int j = 0; j < nblk; ++j) {
       if (j >= kPStages && !ptx::mbar_wait(&pempty[s], ph ^ 1u, limit)) {
-        atomicExch(p.error, 22u);
+        ptx::record_wait_failure(p.error, 22u);
         limit = 1;
       }
       ptx::mbar_arrive_expect_tx(&pfull[s], kPBytes);
@@ -197,7 +197,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
     uint32_t ph = 0;
     for (int k = 0; k < ngroups; ++k) {
       if (!ptx::mbar_wait(&full[pr], ph, limit)) {
-        atomicExch(p.error, 23u);
+        ptx::record_wait_failure(p.error, 23u);
         limit = 1;
       }
       ptx::tc_fence_after();
@@ -230,7 +230,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
       const __half2 dd = __halves2half2(dnext, dnext);
       if (j + 1 < nblk) dnext = nvalid ? __ldg(drow + j + 1) : __float2half(0.f);
       if (!ptx::mbar_wait(&pfull[pst], pph, limit)) {
-        atomicExch(p.error, 24u);
+        ptx::record_wait_failure(p.error, 24u);
         limit = 1;
       }
       uint2 wv[kStepsPerBlock];
@@ -243,7 +243,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
 #pragma unroll
       for (int t2 = 0; t2 < kStepsPerBlock / G; ++t2) {
         if (round > 0 && !ptx::mbar_wait(&empty[pr], (uint32_t)((round - 1) & 1), limit)) {
-          atomicExch(p.error, 25u);
+          ptx::record_wait_failure(p.error, 25u);
           limit = 1;
         }
         ptx::tc_fence_after();
@@ -269,7 +269,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__
         if (++pr == PS) { pr = 0; ++round; }
       }
     }
-    if (!ptx::mbar_wait(accf, 0, limit)) atomicExch(p.error, 26u);
+    if (!ptx::mbar_wait(accf, 0, limit)) ptx::record_wait_failure(p.error, 26u);
     ptx::tc_fence_after();
     __syncwarp();
   }
@@ -451,8 +451,8 @@ bool gemm_tc_supported(int fmt, int64_t M, int64_t N, int64_t K) {
 }
 
 size_t gemm_tc_ws_bytes(int fmt, int64_t M, int64_t N, int64_t K, int num_sms) {
-  if (!gemm_tc_supported(fmt, M, N, K)) return 256;
-  return 256 + plan_for(M, N, K, num_sms).scratch;
+  if (!gemm_tc_supported(fmt, M, N, K)) return 0;
+  return plan_for(M, N, K, num_sms).scratch;
 }
 
 cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __half* d, __half* Y,
@@ -483,8 +483,9 @@ cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __
       return cudaErrorInvalidValue;
   }
   TcParams p;
-  p.error = static_cast<unsigned*>(ws);
-  p.scratch = reinterpret_cast<float4*>(static_cast<uint8_t*>(ws) + 256);
+  const cudaError_t ew = wait_status_word(&p.error);
+  if (ew != cudaSuccess) return ew;
+  p.scratch = static_cast<float4*>(ws);
   p.M = M; p.N = N; p.K = K; p.B = K / kBlock;
   p.NB = pl.NB; p.S = pl.S; p.splits = pl.splits;
   if (pl.smem > (size_t)kMaxSmem) return cudaErrorInvalidValue;

@@ -102,12 +102,7 @@ __device__ __forceinline__ void cp_async_cg16(uint32_t dst, const void* src, uin
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                : "memory");
 }
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* a) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
-  return v;
-}
-constexpr int kSpinLimit = 1 << 22;   // ~0.3 s of 64 ns sleeps: far beyond any real wait
+constexpr int kSpinLimit = 1 << 22;   // stamp polls: a 64 ns sleep + an L2 read, ~256 ns each, ~1 s in all
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -367,7 +362,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int m = 0; m < M; ++m)
-            v[k][h][m] = k < nb ? ld_relaxed_u64(p.partials + (size_t)(c0 + k) * kRT * M + (r_local + 8 * h) * M + m)
+            v[k][h][m] = k < nb ? ptx::ld_relaxed_u64(p.partials + (size_t)(c0 + k) * kRT * M + (r_local + 8 * h) * M + m)
                                 : 0ull;
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {
@@ -378,11 +373,8 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
           for (int m = 0; m < M; ++m) {
             unsigned long long x = v[k][h][m];
             const unsigned long long* a = p.partials + (size_t)(c0 + k) * kRT * M + (r_local + 8 * h) * M + m;
-            for (int spin = 0; (x >> 32) != stamp && spin < kSpinLimit; ++spin) {
-              __nanosleep(64);
-              x = ld_relaxed_u64(a);
-            }
-            if ((x >> 32) != stamp) atomicOr(p.error, 1u);
+            x = ptx::wait_stamp(a, x, stamp, kSpinLimit);
+            if ((x >> 32) != stamp) ptx::record_wait_failure(p.error, 11u);
             sum[h][m] += __uint_as_float((unsigned)x);
           }
       }
@@ -518,7 +510,7 @@ struct Layout {
   int T, G, P;
   long long U;
   size_t smem;
-  size_t off_err, off_part, total;
+  size_t off_part, total;
 };
 
 template <int M>
@@ -542,8 +534,7 @@ Layout layout_m(int64_t N, int64_t K, int num_sms) {
   long long per = ceil_div(L.U, G);
   if (per > L.P) per = L.P;
   L.smem = (size_t)C::kRing + (size_t)per * C::kPairBytes;
-  L.off_err = 0;
-  L.off_part = 256;
+  L.off_part = 0;
   L.total = L.off_part + up256((size_t)G * kRT * M * 8);
   return L;
 }
@@ -625,7 +616,8 @@ cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half
   p.partials = reinterpret_cast<unsigned long long*>(w + L.off_part);
   cudaError_t e0 = epoch_slot(ws, &p.epoch, &p.slot);
   if (e0 != cudaSuccess) return e0;
-  p.error = reinterpret_cast<unsigned*>(w + L.off_err);
+  e0 = wait_status_word(&p.error);
+  if (e0 != cudaSuccess) return e0;
   p.N = N; p.K = K; p.B = K / kBlock; p.P = L.P; p.T = L.T; p.G = L.G; p.U = L.U;
   p.k4 = 4; p.k16 = 16; p.k64 = 64;
   cudaError_t e = smem_attribute<M>();

@@ -51,7 +51,7 @@ constexpr int kCtasPerSm = 2;
 constexpr int kSmemBudget = 110 * 1024;         // two CTAs per SM
 constexpr int kABytes = kRows * (kBlock / 4);   // 8 KB packed weights per block and tile
 constexpr float kQMax = 8.0e6f;
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kWaitLimit = 1u << 18;   // mbarrier polls: ~4 us each when pending, ~1 s in all
 constexpr int kMaxSplit = 8;
 
 // activation record of one block: [ks 2][g 4][t NT][lane 32] uint2, then
@@ -194,7 +194,7 @@ i8n_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restrict__ 
       int s = 0, round = 0;
       for (int j = 0; j < nblk; ++j) {
         if (round > 0 && !ptx::mbar_wait(&empty[s], (uint32_t)((round - 1) & 1), limit)) {
-          atomicExch(p.error, 41u);
+          ptx::record_wait_failure(p.error, 41u);
           limit = 1;
         }
         uint8_t* st = smem + (size_t)s * kStage;
@@ -224,7 +224,7 @@ i8n_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restrict__ 
       dn1 = dm1;
       if (j + 2 < nblk) { dm0 = __ldg(dr0 + j + 2); dm1 = __ldg(dr1 + j + 2); }
       if (!ptx::mbar_wait(&full[s], ph, limit)) {
-        atomicExch(p.error, 42u);
+        ptx::record_wait_failure(p.error, 42u);
         limit = 1;
       }
       const uint32_t st = ptx::smem_u32(smem + (size_t)s * kStage);
@@ -370,7 +370,7 @@ NPlan nplan(int64_t M, int64_t N, int64_t K, int num_sms) {
   int sp = 1;
   while (sp < kMaxSplit && sp < B && (int64_t)pl.tiles * (sp * 2) <= (int64_t)num_sms * kCtasPerSm) sp *= 2;
   pl.splits = sp;
-  pl.off_rec = 256;
+  pl.off_rec = 0;
   pl.off_scr = pl.off_rec + (((size_t)B * rec_bytes(pl.NT) + 255) & ~size_t(255));
   pl.total = pl.off_scr + (sp > 1 ? (size_t)pl.tiles * sp * kRows * M * 4 : 0);
   return pl;
@@ -431,7 +431,8 @@ cudaError_t launch_nt(const NPlan& pl, const __half* X, const uint8_t* qs, const
   NParams p;
   p.recs = recs;
   p.scratch = reinterpret_cast<float*>(w + pl.off_scr);
-  p.error = reinterpret_cast<unsigned*>(w);
+  const cudaError_t ew = wait_status_word(&p.error);
+  if (ew != cudaSuccess) return ew;
   p.M = M; p.N = N; p.K = K; p.B = B; p.splits = pl.splits; p.stages = pl.S;
   p.swiglu = swiglu ? 1 : 0;
   cudaLaunchConfig_t cfg = {};

@@ -55,7 +55,7 @@ template <int MP> struct Unit {
   static constexpr int kWBytes = kRT * 64;                 // packed bytes per unit
   static constexpr int kBoxes = kRT / kBoxRows;
 };
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kWaitLimit = 1u << 18;   // mbarrier polls: ~4 us each when pending, ~1 s in all
 constexpr int kSmemBudget = 220 * 1024;
 
 struct Params {
@@ -251,7 +251,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
           for (int e = 0; e < 4; ++e) acc[t][nt][e] = 0.f;
     }
     if (!ptx::mbar_wait(&full[s], ph, limit)) {
-      atomicExch(p.error, 2u);
+      ptx::record_wait_failure(p.error, 2u);
       limit = 1;
     }
     // B fragments: pairs (x_{16G+j}, x_{16G+j+8}) for the 16-groups G = 4c + q
@@ -293,7 +293,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
     if (warp == 0 && lane == 0 && (u - u0) + S < n) {
       // refill this stage with unit u + S once every warp has released it
       if (!ptx::mbar_wait(&empty[s], ph, limit)) {
-        atomicExch(p.error, 1u);
+        ptx::record_wait_failure(p.error, 1u);
         limit = 1;
       }
       issue(s, pb, prt);
@@ -422,7 +422,7 @@ gemv_mma_kernel(const __grid_constant__ CUtensorMap qmap, const __half* __restri
 
 // ---------------------------------------------------------------- host side
 struct Layout {
-  size_t off_err, off_cnt, off_xil, off_bias, off_dt, off_part, total;
+  size_t off_cnt, off_xil, off_bias, off_dt, off_part, total;
   int64_t Npad;
 };
 
@@ -435,8 +435,7 @@ Layout layout_for(int64_t M, int64_t N, int64_t K, int num_sms) {
   const int64_t U = T * B;
   const int64_t G = U < num_sms ? U : num_sms;
   Layout L;
-  L.off_err = 0;
-  L.off_cnt = 256;
+  L.off_cnt = 0;
   L.off_xil = L.off_cnt + up256((size_t)T * 4);
   L.off_bias = L.off_xil + up256((size_t)B * MP * 512);
   L.Npad = T * kRT;
@@ -485,7 +484,8 @@ cudaError_t launch_mp(const __half* X, const uint8_t* qs, const __half* d, __hal
   p.Npad = (int)L.Npad;
   p.partials = reinterpret_cast<float*>(w + L.off_part);
   p.counters = reinterpret_cast<unsigned*>(w + L.off_cnt);
-  p.error = reinterpret_cast<unsigned*>(w + L.off_err);
+  const cudaError_t ew = wait_status_word(&p.error);
+  if (ew != cudaSuccess) return ew;
 
   auto enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -587,9 +587,9 @@ cudaError_t launch_gemv_mma_noalloc(const __half* X, const uint8_t* qs, const __
   if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
   if (gemv_noalloc_scratch_need(M, N, K, num_sms) > kNoAllocScratchBytes) return cudaErrorInvalidValue;
   uint8_t* ws = static_cast<uint8_t*>(g_scratch_addr[dev]);
-  // the tickets (one per 128-row tile, after a 256-byte header in both decode
-  // kernels' layouts) must start at zero; the array keeps the last call's bytes
-  e = cudaMemsetAsync(ws + 256, 0, up256((size_t)ceil_div(N, 128) * 4), s);
+  // the tickets (one per 128-row tile, at the head of the layout) must start
+  // at zero; the array keeps the last call's bytes
+  e = cudaMemsetAsync(ws, 0, up256((size_t)ceil_div(N, 128) * 4), s);
   if (e != cudaSuccess) return e;
   return launch_gemv_mma(TRI_TQ2, X, qs, d, Y, M, N, K, ws, num_sms, s);
 }

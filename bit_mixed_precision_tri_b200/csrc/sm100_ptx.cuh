@@ -52,6 +52,32 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* a) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(a) : "memory");
+  return v;
+}
+
+// Bounded wait for a stamped 64-bit word written by another thread block: the
+// high half carries the writer's stamp.  `x` is a value already read from `a`;
+// polls (64 ns sleeps in between) until the stamp matches or `limit` polls
+// have gone by, and returns the last value read.
+__device__ __forceinline__ unsigned long long wait_stamp(const unsigned long long* a,
+                                                         unsigned long long x, unsigned stamp,
+                                                         int limit) {
+  for (int spin = 0; (unsigned)(x >> 32) != stamp && spin < limit; ++spin) {
+    __nanosleep(64);
+    x = ld_relaxed_u64(a);
+  }
+  return x;
+}
+
+// A bounded wait gave up: keep the first non-zero code in the device's wait
+// status word (later codes are dropped so the first cause stays readable).
+__device__ __forceinline__ void record_wait_failure(unsigned* word, unsigned code) {
+  atomicCAS(word, 0u, code);
+}
+
 // 2-D tiled TMA load global -> shared, completion on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar, uint64_t policy) {

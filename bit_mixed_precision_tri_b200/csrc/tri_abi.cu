@@ -1,7 +1,8 @@
 // The C ABI (include/tri.h): host-side validation and dispatch.
 //
 // Every entry point checks its arguments before enqueuing anything, launches
-// on the caller's stream, never allocates and never synchronizes.
+// on the caller's stream and never allocates; only tri_wait_status
+// synchronizes (it exists to read a device-side result).
 #include <mutex>
 
 #include "tri_internal.cuh"
@@ -345,6 +346,26 @@ tri_status tri_gemm_tq2_noalloc(const uint16_t* X, const uint8_t* qs, const uint
   return from_cuda(tri::launch_gemv_mma_noalloc(
       reinterpret_cast<const __half*>(X), qs, reinterpret_cast<const __half*>(d),
       reinterpret_cast<__half*>(Y), (int)M, (int)N, (int)K, di.sms, static_cast<cudaStream_t>(stream)));
+}
+
+tri_status tri_wait_status(uint32_t* code, int clear, void* stream) {
+  if (!code) return TRI_ERR_INVALID_ARG;
+  DevInfo di;
+  tri_status st = device_info(&di);
+  if (st != TRI_OK) return st;
+  unsigned c = 0;
+  st = from_cuda(tri::read_wait_status(&c, clear != 0, static_cast<cudaStream_t>(stream)));
+  if (st == TRI_OK) *code = c;
+  return st;
+}
+
+tri_status tri_selftest_wait_timeout(int which, void* scratch, void* stream) {
+  if ((which != 0 && which != 1) || !scratch) return TRI_ERR_INVALID_ARG;
+  if (!aligned(scratch, 8)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  tri_status st = device_info(&di);
+  if (st != TRI_OK) return st;
+  return from_cuda(tri::launch_expire_wait(which, scratch, static_cast<cudaStream_t>(stream)));
 }
 
 tri_status tri_gemm_tq2(const uint16_t* X, const uint8_t* qs, const uint16_t* d, uint16_t* Y,

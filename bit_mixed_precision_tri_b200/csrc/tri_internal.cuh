@@ -76,6 +76,19 @@ cudaError_t launch_gemm_tc(int fmt, const __half* X, const uint8_t* qs, const __
                            __half* Y, int M, int N, int K, void* ws, int num_sms,
                            cudaStream_t s);
 
+// ---- device wait status (status.cu) ----------------------------------------
+// codes recorded by a bounded wait that ran out; the values name the wait:
+// 1-2 gemv_mma.cu, 11 gemv_i8.cu, 21-26 gemm_tc.cu, 41-42 gemv_i8n.cu
+constexpr unsigned kSelfTestMbarCode = 90;
+constexpr unsigned kSelfTestStampCode = 91;
+// the current device's status word (device address)
+cudaError_t wait_status_word(unsigned** out);
+// synchronizes `s`, then copies the word to *code and optionally zeroes it
+cudaError_t read_wait_status(unsigned* code, bool clear, cudaStream_t s);
+// a one-block kernel whose wait (0: mbarrier, 1: stamped word) runs out;
+// `scratch` is 8 device bytes the stamped word lives in
+cudaError_t launch_expire_wait(int which, void* scratch, cudaStream_t s);
+
 // ---- small helpers ---------------------------------------------------------
 __host__ __device__ inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

@@ -19,15 +19,17 @@
  *    X is M x K fp16 row-major, Y is M x N fp16 row-major.  K must be a
  *    positive multiple of 256 (one block = 256 consecutive weights of a row).
  *  - Every data pointer is a DEVICE pointer, allocated and owned by the
- *    caller.  The library allocates nothing and never synchronizes the host;
- *    all work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
- *    stream) in call order.
+ *    caller.  The library allocates nothing and, except in tri_wait_status,
+ *    never synchronizes the host; all work is enqueued on `stream` (a
+ *    cudaStream_t; NULL = legacy default stream) in call order.
  *  - fp16 tensors are passed as uint16_t bit patterns (IEEE binary16).
  *  - Arguments are validated on the host before anything is enqueued; a
  *    non-OK status means nothing was launched.  A launch failure reported by
  *    the CUDA runtime returns TRI_ERR_CUDA.  No kernel traps or asserts:
  *    data errors (non-finite weights, invalid packed codes) are reported
- *    through device-side results described per function.
+ *    through device-side results described per function, and every wait of
+ *    one thread block on another or on an asynchronous copy is bounded and
+ *    reports through the device wait status word (tri_wait_status).
  *  - Buffers given to one call must not overlap unless stated.
  *
  * Packed formats (readings of the pages, fixed by this library)
@@ -252,6 +254,33 @@ TRI_API size_t tri_gemm_swiglu_workspace_bytes(int format, int64_t M, int64_t F,
 TRI_API tri_status tri_gemm_swiglu(int format, int path, const uint16_t* X, const uint8_t* qs,
                                    const uint16_t* d, uint16_t* Y, int64_t M, int64_t F, int64_t K,
                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Device wait status.  The GEMM kernels wait on asynchronous copies, on the
+ * tensor-core pipeline and on partial sums of other thread blocks; each such
+ * wait gives up after an iteration limit far beyond any wait a healthy call
+ * sees (a second or more).  A wait that gives up stores a non-zero code in a
+ * 32-bit word the library keeps on each device (the first code stays until
+ * cleared; later ones are dropped), lets the kernel drain and return, and
+ * leaves that call's output unspecified.  Codes name the wait: 1-2 and 11
+ * the decode kernels (M <= 2), 41-42 the integer kernel for 3 <= M <= 16,
+ * 21-26 the tcgen05 kernel (M > 16), 90-91 tri_selftest_wait_timeout.
+ *
+ * tri_wait_status: waits for `stream` to finish (cudaStreamSynchronize),
+ *   then stores the current device's word in *code (0 = no wait has given up
+ *   since the last clear) and, if `clear` is non-zero, zeroes it.  The one
+ *   entry point that synchronizes the host.  Word reads and clears race with
+ *   kernels of this library still running on other streams.
+ * tri_selftest_wait_timeout: enqueues on `stream` one kernel whose wait can
+ *   never complete, through the same bounded routines the GEMM kernels use:
+ *   which = 0 waits on an mbarrier phase nothing arrives on (code 90),
+ *   which = 1 on a stamped word nothing writes (code 91; the word is the
+ *   first 8 bytes of `scratch`, device memory, 8-byte aligned, zeroed by the
+ *   call).  The wait runs out within about a second, records its code and
+ *   returns; nothing faults.  It lets a caller check the detection path.
+ * ---------------------------------------------------------------------- */
+TRI_API tri_status tri_wait_status(uint32_t* code, int clear, void* stream);
+TRI_API tri_status tri_selftest_wait_timeout(int which, void* scratch, void* stream);
 
 /* Kernel that tri_gemm would launch for this call under TRI_PATH_AUTO
  * (one of tri_gemm_path), or -1 if the shape is invalid. */

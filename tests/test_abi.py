@@ -86,3 +86,11 @@ def test_auto_path_and_workspace_query(L):
             p = L.tri_gemm_auto_path(fmt, M, 4096, 4096)
             assert p in (1, 2, 3, 4)
             assert L.tri_gemm_workspace_bytes(fmt, M, 4096, 4096) >= 256
+
+
+def test_wait_status_entry_points_reject_bad_arguments(L):
+    assert L.tri_wait_status(None, 1, None) == 1                       # null code pointer
+    assert L.tri_selftest_wait_timeout(2, FAKE, None) == 1             # no such wait
+    assert L.tri_selftest_wait_timeout(-1, FAKE, None) == 1
+    assert L.tri_selftest_wait_timeout(0, None, None) == 1             # null scratch
+    assert L.tri_selftest_wait_timeout(1, FAKE + 4, None) == 3         # scratch not 8-byte aligned
