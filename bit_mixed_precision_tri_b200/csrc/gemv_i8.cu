@@ -281,27 +281,28 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
           const float inv = amax > 0.f ? kQMax / amax : 0.f;
-          int dg[3][8];
+          // Balanced base-256 digits of q, as bytes: with u = q + 0x808080
+          // (in [0, 2^24) for |q| <= 8e6), byte i of u is digit i + 128, so
+          // byte i of u ^ 0x808080 is digit i as a signed byte (byte 0 the
+          // lowest digit, byte 2 the highest).
+          uint32_t dg[8];
           int sum = 0;
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int q = __float2int_rn(xv[e] * inv);   // |q| <= 8e6 < 2^23
             sum += q;
-            const int lo = ((q + 128) & 255) - 128;
-            const int r1 = (q - lo) >> 8;
-            const int mid = ((r1 + 128) & 255) - 128;
-            dg[0][e] = (r1 - mid) >> 8;
-            dg[1][e] = mid;
-            dg[2][e] = lo;
+            dg[e] = ((uint32_t)q + 0x808080u) ^ 0x808080u;
           }
+          // level lv = column 3m + lv holds digit 2 - lv (the highest first);
+          // the two bytes of field g are elements g and g + 4
 #pragma unroll
           for (int lv = 0; lv < 3; ++lv)
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const int off = ((f_p * 2 + (g >> 1)) * C::kBSlots + (3 * m + lv) * 4 + f_tig) * 16 +
                               ((g & 1) * 2 + f_r) * 4 + 2 * half;
-              *reinterpret_cast<uint16_t*>(rec + off) =
-                  (uint16_t)((dg[lv][g] & 255) | ((dg[lv][g + 4] & 255) << 8));
+              const uint32_t sel = (uint32_t)(2 - lv) | ((uint32_t)(6 - lv) << 4);
+              *reinterpret_cast<uint16_t*>(rec + off) = (uint16_t)__byte_perm(dg[g], dg[g + 4], sel);
             }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);

@@ -105,22 +105,27 @@ i8n_prep_kernel(const __half* __restrict__ X, int M, int K, uint8_t* __restrict_
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
   const float inv = amax > 0.f ? kQMax / amax : 0.f;
-  // digits of element 4 j + g, level l, packed per (l, g) over j
-  uint32_t wd[3][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}, {0, 0, 0, 0}};
+  // Balanced base-256 digits of q as bytes: with u = q + 0x808080 (in
+  // [0, 2^24) for |q| <= 8e6), byte i of u ^ 0x808080 is digit i as a signed
+  // byte.  Level l (0 = highest digit) of element 4 j + g goes to byte j of
+  // wd[l][g].
+  uint32_t dg[16];
   int sum = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const int q = __float2int_rn(xv[i] * inv);         // |q| <= 8e6 < 2^23
     sum += q;
-    const int lo = ((q + 128) & 255) - 128;
-    const int r1 = (q - lo) >> 8;
-    const int mid = ((r1 + 128) & 255) - 128;
-    const int hi = (r1 - mid) >> 8;
-    const int j = i >> 2, g = i & 3;
-    wd[0][g] |= (uint32_t)(hi & 255) << (8 * j);
-    wd[1][g] |= (uint32_t)(mid & 255) << (8 * j);
-    wd[2][g] |= (uint32_t)(lo & 255) << (8 * j);
+    dg[i] = ((uint32_t)q + 0x808080u) ^ 0x808080u;
   }
+  uint32_t wd[3][4];
+#pragma unroll
+  for (int l = 0; l < 3; ++l)
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t sel = (uint32_t)(2 - l) | ((uint32_t)(6 - l) << 4);
+      const uint32_t lo = __byte_perm(dg[g], dg[4 + g], sel), hi = __byte_perm(dg[8 + g], dg[12 + g], sel);
+      wd[l][g] = __byte_perm(lo, hi, 0x5410);
+    }
 #pragma unroll
   for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
   if (m < 8 * NT / 3) {                        // rows that have columns (all of them when NT = 6)
