@@ -278,8 +278,9 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
           float amax = 0.f;
 #pragma unroll
           for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(xv[e]));
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+          // |x| >= 0: the bit patterns order like the values, so one integer
+          // warp reduction gives the block maximum
+          amax = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax)));
           const float inv = amax > 0.f ? kQMax / amax : 0.f;
           // Balanced base-256 digits of q, as bytes: with u = q + 0x808080
           // (in [0, 2^24) for |q| <= 8e6), byte i of u is digit i + 128, so
@@ -304,8 +305,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
               const uint32_t sel = (uint32_t)(2 - lv) | ((uint32_t)(6 - lv) << 4);
               *reinterpret_cast<uint16_t*>(rec + off) = (uint16_t)__byte_perm(dg[g], dg[g + 4], sel);
             }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+          sum = __reduce_add_sync(0xFFFFFFFFu, sum);
           if (lane == 0) {
             sc[m] = amax > 0.f ? (amax / kQMax) * (1.f / 64.f) : 0.f;   // s_b / 64
             sc[M + m] = 64.f * (float)sum;                              // 64 sum_k x^_k
