@@ -65,11 +65,16 @@ cudaError_t read_wait_status(unsigned* code, bool clear, cudaStream_t s) {
   unsigned* w = nullptr;
   cudaError_t e = wait_status_word(&w);
   if (e != cudaSuccess) return e;
-  e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return e;
-  e = cudaMemcpy(code, w, sizeof(unsigned), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess || !clear) return e;
-  return cudaMemset(w, 0, sizeof(unsigned));
+  // read (and clear) in the stream's order, then wait: the word seen is the
+  // one left by the work enqueued on `s` before this call, and the clear is
+  // complete before returning
+  unsigned v = 0;
+  e = cudaMemcpyAsync(&v, w, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && clear) e = cudaMemsetAsync(w, 0, sizeof(unsigned), s);
+  const cudaError_t es = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = es;
+  if (e == cudaSuccess) *code = v;
+  return e;
 }
 
 cudaError_t launch_expire_wait(int which, void* scratch, cudaStream_t s) {

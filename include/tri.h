@@ -266,11 +266,12 @@ TRI_API tri_status tri_gemm_swiglu(int format, int path, const uint16_t* X, cons
  * the decode kernels (M <= 2), 41-42 the integer kernel for 3 <= M <= 16,
  * 21-26 the tcgen05 kernel (M > 16), 90-91 tri_selftest_wait_timeout.
  *
- * tri_wait_status: waits for `stream` to finish (cudaStreamSynchronize),
- *   then stores the current device's word in *code (0 = no wait has given up
- *   since the last clear) and, if `clear` is non-zero, zeroes it.  The one
- *   entry point that synchronizes the host.  Word reads and clears race with
- *   kernels of this library still running on other streams.
+ * tri_wait_status: reads the current device's word in `stream` order (after
+ *   the work already enqueued there), zeroes it there if `clear` is
+ *   non-zero, waits for the stream to finish (cudaStreamSynchronize) and
+ *   stores the value read in *code (0 = no wait has given up since the last
+ *   clear).  The one entry point that synchronizes the host.  Word reads and
+ *   clears race with kernels of this library running on other streams.
  * tri_selftest_wait_timeout: enqueues on `stream` one kernel whose wait can
  *   never complete, through the same bounded routines the GEMM kernels use:
  *   which = 0 waits on an mbarrier phase nothing arrives on (code 90),
