@@ -120,26 +120,32 @@ def auto_path(fmt, M: int, N: int, K: int) -> int:
 
 class Workspace:
     """Device scratch for tri_gemm, grown on demand.  Its contents between
-    calls do not matter; calls that share one must be ordered (one stream)."""
+    calls do not matter; calls that share one must be ordered (one stream).
+    A buffer that grows is allocated on the stream of the call that needs it,
+    so the allocator frees the old one in that stream's order."""
 
     def __init__(self, device=None):
         self.device = torch.device(device or "cuda")
         self.buf = None
 
-    def get(self, nbytes: int) -> torch.Tensor:
+    def get(self, nbytes: int, stream=None) -> torch.Tensor:
         if self.buf is None or self.buf.numel() < nbytes:
-            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            with torch.cuda.stream(stream):          # a no-op for stream=None
+                self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
         return self.buf
 
 
 _default_ws = {}
 
 
-def _workspace_for(device) -> Workspace:
-    key = torch.device(device)
-    if key not in _default_ws:
-        _default_ws[key] = Workspace(key)
-    return _default_ws[key]
+def _workspace_for(device, stream_handle: int) -> Workspace:
+    """The default workspace of (device, stream): calls on different streams
+    never share scratch, calls on one stream are ordered by it."""
+    key = (torch.device(device), int(stream_handle))
+    ws = _default_ws.get(key)
+    if ws is None:
+        ws = _default_ws[key] = Workspace(key[0])
+    return ws
 
 
 def gemm(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, N: int, K: int, fmt="tq2",
@@ -161,8 +167,8 @@ def gemm(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, N: int, K: int, fmt
         if not (out.is_cuda and out.is_contiguous()):
             raise ValueError("out must be a contiguous CUDA tensor")
         Y = out
-    ws = (workspace or _workspace_for(X.device)).get(gemm_workspace_bytes(f, M, N, K))
     s = stream.cuda_stream if stream is not None else _stream(X.device)
+    ws = (workspace or _workspace_for(X.device, s)).get(gemm_workspace_bytes(f, M, N, K), stream)
     st = _lib.lib().tri_gemm(f, int(path), X.data_ptr(), qs.data_ptr(), d.data_ptr(), Y.data_ptr(),
                              M, N, K, ws.data_ptr(), ws.numel(), s)
     if st:
@@ -208,8 +214,9 @@ def gemm_swiglu(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, F: int, K: i
             raise ValueError("out must be a contiguous CUDA tensor")
         Y = out
     L = _lib.lib()
-    ws = (workspace or _workspace_for(X.device)).get(max(int(L.tri_gemm_swiglu_workspace_bytes(f, M, F, K)), 256))
     s = stream.cuda_stream if stream is not None else _stream(X.device)
+    ws = (workspace or _workspace_for(X.device, s)).get(
+        max(int(L.tri_gemm_swiglu_workspace_bytes(f, M, F, K)), 256), stream)
     st = L.tri_gemm_swiglu(f, int(path), X.data_ptr(), qs.data_ptr(), d.data_ptr(), Y.data_ptr(),
                            M, F, K, ws.data_ptr(), ws.numel(), s)
     if st:
