@@ -43,6 +43,9 @@ Parity pins for every function live in tests/test_oracle.py.
 """
 from __future__ import annotations
 
+import itertools
+import math
+
 import numpy as np
 
 BLOCK = 256          # weights per block [TLS "Fast inference on CPUs"]
@@ -54,24 +57,19 @@ TQ1_GROUPS = 51       # full five-trit groups per block (255 trits)
 # --------------------------------------------------------------------------
 # a1: absmean scale  [TLS "The model" step 1; SPC "Architecture"]
 # --------------------------------------------------------------------------
-def exact_abs_sum_scaled(W: np.ndarray) -> int:
-    """Return sum|W| exactly, as an integer count of 2**-149 (float32 ulps).
+def abs_sum_rn64(W: np.ndarray) -> float:
+    """RN64(sum |W|): the exact sum of the absolute values, rounded once to
+    the nearest double.
 
-    Every finite float32 is m * 2**(e-150) with a 24-bit integer m (implicit
-    bit included for normal numbers) and e = max(biased exponent, 1), so it is
-    an integer multiple of 2**-149.  Summing the integers is exact.
+    math.fsum (Shewchuk's exact partials) returns the correctly rounded sum
+    of its arguments; every float32 |w| is exactly a double, so this is the
+    plain definition of reading R1 with no reduction order in it.  The values
+    are fed in chunks only to bound memory; fsum sees one stream.
     """
-    a = np.ascontiguousarray(W, dtype=np.float32).reshape(-1)
-    bits = a.view(np.uint32) & np.uint32(0x7FFFFFFF)      # |w|
-    e = (bits >> np.uint32(23)).astype(np.int64)
-    m = (bits & np.uint32(0x7FFFFF)).astype(np.int64)
-    m = m + np.where(e > 0, np.int64(1) << 23, np.int64(0))
-    e = np.maximum(e, 1)
-    total = 0
-    for ex in np.unique(e):
-        # |w| = m * 2**(ex - 150) = m * 2**(ex - 1) * 2**-149
-        total += int(m[e == ex].sum(dtype=np.int64)) << int(ex - 1)
-    return total
+    a = np.abs(np.ascontiguousarray(W, dtype=np.float32).reshape(-1))
+    chunk = 1 << 22
+    return math.fsum(itertools.chain.from_iterable(
+        a[i:i + chunk].astype(np.float64).tolist() for i in range(0, a.size, chunk)))
 
 
 def absmean_gamma(W: np.ndarray, eps: float) -> np.float32:
@@ -82,11 +80,10 @@ def absmean_gamma(W: np.ndarray, eps: float) -> np.float32:
     a = np.ascontiguousarray(W, dtype=np.float32)
     if a.size == 0 or not np.all(np.isfinite(a)):
         return np.float32(np.nan)
-    s_scaled = exact_abs_sum_scaled(a)
-    s64 = s_scaled / (1 << 149)          # Python int / int: correctly rounded
-    mean64 = s64 / float(a.size)          # IEEE double division
-    g64 = mean64 + float(np.float32(eps))  # IEEE double addition
-    return np.float32(g64)                 # round to nearest float32
+    s64 = abs_sum_rn64(a)                   # RN64(S)
+    mean64 = s64 / float(a.size)            # IEEE double division
+    g64 = mean64 + float(np.float32(eps))   # IEEE double addition
+    return np.float32(g64)                  # round to nearest float32
 
 
 # --------------------------------------------------------------------------

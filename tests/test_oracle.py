@@ -1,6 +1,7 @@
 """Pins for the CPU oracle: each check compares it with something other than
 itself -- values printed on the pages, closed forms, independent library
-routines (math.fsum), exact rational brute force, and a second decoder.
+routines, exact rational arithmetic (Fractions), brute force, and a second
+decoder.
 
 Pages: "Scaling Laws and Efficient Inference for Ternary Language Models"
 (sections "The model", "Packing ternary weights", "Fast inference on CPUs",
@@ -27,11 +28,16 @@ def _gold(name):
 
 
 # ---------------------------------------------------------------- a1 gamma
+def _fraction_abs_sum(w):
+    """Exact rational sum of |w| (Python Fractions), independent of math.fsum."""
+    return sum((Fraction(abs(float(v))) for v in np.asarray(w, np.float32).reshape(-1)), Fraction(0))
+
+
 @pytest.mark.parametrize("seed", range(6))
-def test_exact_sum_matches_fsum(seed):
-    """RN64 of the oracle's exact sum equals math.fsum (correctly rounded)."""
+def test_abs_sum_is_the_correctly_rounded_exact_sum(seed):
+    """RN64 of the exact sum: float(Fraction) rounds a rational correctly."""
     rng = np.random.default_rng(seed)
-    n = 5000
+    n = 3000
     kind = seed % 3
     if kind == 0:
         w = rng.standard_normal(n) * 0.02
@@ -41,16 +47,30 @@ def test_exact_sum_matches_fsum(seed):
     else:             # large and tiny values mixed: rounding depends on tiny ones
         w = np.where(rng.random(n) < 0.5, 1e30, 1e-30) * rng.standard_normal(n)
     w = w.astype(np.float32)
-    exact = O.exact_abs_sum_scaled(w) / (1 << 149)
-    ref = math.fsum(abs(float(v)) for v in w)
-    assert exact == ref
+    assert O.abs_sum_rn64(w) == float(_fraction_abs_sum(w))
 
 
-def test_exact_sum_denormal_and_powers():
+def test_abs_sum_denormal_and_powers():
     w = np.array([np.float32(2.0 ** -149), np.float32(2.0 ** -126), np.float32(-1.0),
                   np.float32(3.0), np.float32(2.0 ** 100)], dtype=np.float32)
-    S = O.exact_abs_sum_scaled(w)
-    assert Fraction(S, 1 << 149) == Fraction(1, 1 << 149) + Fraction(1, 1 << 126) + 4 + (1 << 100)
+    exact = Fraction(1, 1 << 149) + Fraction(1, 1 << 126) + 4 + (1 << 100)
+    assert O.abs_sum_rn64(w) == float(exact) == 2.0 ** 100
+
+
+def test_abs_sum_is_not_a_running_float_sum():
+    """1 + 2^-53 + 2^-53: a left-to-right double sum loses both small terms
+    (each addition is a tie, rounded to even), the exact sum is 1 + 2^-52."""
+    w = np.array([1.0, 2.0 ** -53, -(2.0 ** -53)], dtype=np.float32)
+    naive = 0.0
+    for v in w.tolist():
+        naive += abs(v)
+    assert naive == 1.0
+    assert O.abs_sum_rn64(w) == 1.0 + 2.0 ** -52
+    # reversed order: a running sum would now be exact; the oracle is order-free
+    assert O.abs_sum_rn64(w[::-1].copy()) == 1.0 + 2.0 ** -52
+    # gamma from it: mean = (1 + 2^-52)/4 in double, then float32
+    g = O.absmean_gamma(np.append(w, np.float32(0.0)), 0.0)
+    assert g == np.float32((1.0 + 2.0 ** -52) / 4)
 
 
 def test_gamma_hand_example():
@@ -108,6 +128,38 @@ def test_ternarize_matches_scalar_python():
         q = float(np.float32(w / g))   # double quotient of floats, rounded once to f32
         q = max(-1.0, min(1.0, q))
         assert round(q) == t           # Python round(): half to even
+
+
+def test_ternarize_nan_quotient_is_zero_and_infinities_clip():
+    """Reading R2 at its edges, by IEEE rules written out by hand:
+    NaN / g is NaN -> 0; +-inf / g = +-inf -> clip -> +-1; with gamma = 0,
+    0 / 0 is NaN -> 0 and w / 0 = +-inf -> +-1."""
+    W = np.array([np.nan, np.inf, -np.inf, 0.3, -0.04, 0.0], dtype=np.float32)
+    assert O.ternarize(W, np.float32(0.1)).tolist() == [0, 1, -1, 1, 0, 0]
+    W = np.array([0.0, -0.0, 1e-30, -2.0], dtype=np.float32)
+    assert O.ternarize(W, np.float32(0.0)).tolist() == [0, 0, 1, -1]
+    # a NaN gamma (what absmean_gamma returns for non-finite W) zeroes every trit
+    assert O.ternarize(np.array([1.0, -1.0, 0.5], np.float32), np.float32(np.nan)).tolist() == [0, 0, 0]
+
+
+def test_invalid_trits_counted_and_packed_as_zero():
+    """Reading R7 for packing: values outside {-1, 0, 1} are counted, packed
+    as the zero weight (field value 1, i.e. d' = 0 + 1)."""
+    t = np.zeros((2, 256), dtype=np.int8)
+    t[0, :6] = [1, -1, 0, 2, -2, 127]
+    t[1, 255] = -128
+    assert O.invalid_trit_count(t) == 4
+    assert O.invalid_trit_count(np.array([-1, 0, 1], np.int8)) == 0
+    qs2, _ = O.pack_tq2(t, 1.0)
+    # byte 0: fields 2,0,1,1 (t = 1,-1,0,0); byte 1: fields 1,1,1,1 (invalid -> 0, 127 -> 0, then zeros)
+    assert int(qs2[0, 0]) == 2 | (0 << 2) | (1 << 4) | (1 << 6)
+    assert int(qs2[0, 1]) == 0b01010101
+    assert int(qs2[1, 63]) == 0b01010101
+    qs1, _ = O.pack_tq1(t, 1.0)
+    # first five-trit group of row 0: (1,-1,0,2->0,-2->0) -> digits 2,0,1,1,1 -> N5 = 162+0+9+3+1 = 175
+    assert int(qs1[0, 0]) == (175 * 256 + 242) // 243
+    # row 1, block's last byte: trit 255 (-128 -> 0) then four zero trits -> digits 1,1,1,1,1 -> N5 = 121
+    assert int(qs1[1, 51]) == (121 * 256 + 242) // 243
 
 
 # ---------------------------------------------------------------- a3 TQ2
