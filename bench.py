@@ -7,8 +7,11 @@
 One step = one pass of the ternary linear layers of the workload over one
 batch of synthetic activations (weights are prepared once: at inference
 only the ternary weights and their scales are kept).  The default
-workload is the single-layer decode GEMV set of a LLaMA-7B-like model
-(W in {4096x4096, 11008x4096, 4096x11008}, M = 1, TQ2).  Weights are
+workload is the decode GEMV of the 70B-like down projection (W 8192x28672,
+M = 1, TQ2), the shape the memory-bound target is stated on; the same line
+carries, under "targets", the compute-regime shape (W 8192x8192, M = 256,
+TQ2) and the LLaMA-7B-like single-layer decode set (W in {4096x4096,
+11008x4096, 4096x11008}, M = 1), each timed the same way.  Weights are
 absmean-ternarized from N(0, 0.02) latent weights by this library, then
 cloned into enough rotating copies that every timed step reads weights that
 are not in L2 (the copies total > 3x the L2 size).  The timed region is one
@@ -400,6 +403,36 @@ def measure_cublas_fp16(w, device, steps, warmup):
             "weight_copies": copies}
 
 
+TARGET_WORKLOADS = ("square_8192_m256", "llama7b_decode_m1")
+
+
+def measure_targets(args, rank, world, device):
+    """The other stated shapes, each timed like the main line (one CUDA graph
+    of K steps over rotating weight copies larger than L2), with its own
+    roofline; the compute-regime shape reports its tensor fraction against
+    both the burst and the sustained measured bf16/fp16 peak."""
+    out = {}
+    peaks, _ = load_peaks()
+    for name in TARGET_WORKLOADS:
+        a = argparse.Namespace(**vars(args))
+        a.steps, a.warmup = min(args.steps, 20), max(3, min(args.warmup, 5))
+        w = workload_from_args(name)
+        r = run_ours(a, rank, world, device, w=w)
+        roof = dict(r["roofline"])
+        if roof["bound"] == "tensor":
+            roof["frac_of_sustained"] = roof["achieved"] / peaks["bf16_tflops_sustained"]
+            roof["peak_sustained"] = peaks["bf16_tflops_sustained"]
+        t = {"value": r["value"], "unit": r["unit"], "ms_per_step": r["ms_per_step"],
+             "steps": a.steps, "warmup": a.warmup, "config": r["config"], "roofline": roof,
+             "e2e": r["e2e"], "gpu_launches": r["gpu_launches"], "clocks": r["clocks"]}
+        if not args.no_cublas:
+            cb = measure_cublas_fp16(w, device, a.steps, a.warmup)
+            cb["speedup_of_ternary"] = cb["ms_per_step"] / r["ms_per_step"]
+            t["cublas_fp16"] = cb
+        out[name] = t
+    return out
+
+
 # ------------------------------------------------------------------ other rows
 def measure_rows(device, N=28672, K=8192, reps=5):
     """Time the offline rows of the path (absmean, ternarize, pack, unpack) on
@@ -452,10 +485,26 @@ def measure_rows(device, N=28672, K=8192, reps=5):
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_sample(w, budget_s=12.0):
+def blas_threads() -> int:
+    """Threads of the BLAS pool that numpy's float64 matmul (the oracle's
+    block products) runs on."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return 1
+
+
+def oracle_sample(w, budget_s=12.0, threads=None):
     """Time the CPU oracle (as it stands) on a bounded sample of the workload:
-    whole layers (unpack + fp64 GEMM) until ~budget_s of CPU work; returns
-    (value in the workload's unit, description, threads)."""
+    whole layers (unpack + fp64 GEMM) until ~budget_s of CPU work.  With
+    ``threads`` the BLAS pool is limited to that many threads for the timing.
+    Returns a dict: value (the workload's unit), unit, sample description,
+    threads used, elapsed seconds."""
+    import contextlib
     from bit_mixed_precision_tri_b200 import inputs
     from oracle import tri_oracle as O
     M, fmt = w["M"], w["fmt"]
@@ -468,27 +517,32 @@ def oracle_sample(w, budget_s=12.0):
         qs, d = O.pack(fmt, t, np.array([g], np.float32))
         X = inputs.activations(M, K, 6 + M + seed).numpy()
         prepared.append((rows, K, qs, d, X))
-    done_bytes = done_flops = 0.0
-    t0 = time.perf_counter()
-    n = 0
-    while True:
-        for rows, K, qs, d, X in prepared:
-            O.gemm_packed_f64(fmt, X, qs, d, rows, K)
-            done_bytes += algo_bytes(fmt, M, rows, K)
-            done_flops += 2.0 * M * rows * K
-        n += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
+    limit = contextlib.nullcontext()
+    if threads is not None:
+        try:
+            from threadpoolctl import threadpool_limits
+            limit = threadpool_limits(limits=threads, user_api="blas")
+        except Exception:
+            pass
+    with limit:
+        used = blas_threads()
+        done_bytes = done_flops = 0.0
+        t0 = time.perf_counter()
+        n = 0
+        while True:
+            for rows, K, qs, d, X in prepared:
+                O.gemm_packed_f64(fmt, X, qs, d, rows, K)
+                done_bytes += algo_bytes(fmt, M, rows, K)
+                done_flops += 2.0 * M * rows * K
+            n += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
     val = done_bytes / dt / 1e9 if unit == "GB/s" else done_flops / dt / 1e12
     desc = (f"{n} passes over the first min(N, 2048) rows of each layer "
             f"({'+'.join(str(min(N, 2048)) + 'x' + str(K) for N, K in w['layers'])}), "
-            f"unpack + float64 GEMM, {dt:.1f} s")
-    try:
-        threads = len(os.sched_getaffinity(0))
-    except Exception:
-        threads = os.cpu_count()
-    return val, unit, desc, threads
+            f"unpack + float64 GEMM (numpy, BLAS on {used} thread(s)), {dt:.1f} s")
+    return {"value": val, "unit": unit, "sample": desc, "threads": used, "elapsed_s": dt}
 
 
 def run_reference(args, rank, world):
@@ -496,22 +550,25 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     budget = max(3.0, 60.0 / max(args.steps + args.warmup, 1))
-    vals = []
+    samples = []
     for i in range(args.warmup + args.steps):
-        v, unit, desc, threads = oracle_sample(w, budget_s=budget)
+        r = oracle_sample(w, budget_s=budget)
         if i >= args.warmup:
-            vals.append(v)
-    value = statistics.mean(vals)
+            samples.append(r)
+    value = statistics.mean(r["value"] for r in samples)
+    unit = samples[0]["unit"]
     return {
         "impl": "reference",
         "metric": "TQ2/TQ1 ternary GEMM: HBM GB/s (M<=16) and TFLOP/s (M>=64) vs roofline",
         "value": value, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": budget * 1e3, "higher_is_better": True, "scaling": "weak",
+        # measured: the mean wall time of one step (one bounded oracle sample)
+        "ms_per_step": statistics.mean(r["elapsed_s"] for r in samples) * 1e3,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w["name"], "layers_NxK": [f"{N}x{K}" for N, K in w["layers"]],
                    "M": w["M"], "format": w["fmt"]},
-        "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": samples[0]["threads"], "kind": "oracle",
+                         "sample": samples[0]["sample"]},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -571,12 +628,14 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="llama7b_decode_m1", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="down_8192x28672_m1", choices=sorted(WORKLOADS))
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--fmt", default=None, choices=[None, "tq2", "tq1"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip timing the offline rows")
     ap.add_argument("--no-cublas", action="store_true", help="skip the cuBLAS fp16 comparison")
+    ap.add_argument("--no-targets", action="store_true",
+                    help="skip the extra target workloads of the default line")
     ap.add_argument("--sweep", action="store_true",
                     help="print one line per batch-sweep, block and format-stress workload")
     args = ap.parse_args()
@@ -608,13 +667,19 @@ def main():
             cb = measure_cublas_fp16(w, device, args.steps, args.warmup)
             cb["speedup_of_ternary"] = cb["ms_per_step"] / res["ms_per_step"]
             res["cublas_fp16"] = cb
+        if not args.no_targets and args.workload == "down_8192x28672_m1" and args.M is None \
+                and args.fmt is None:
+            res["targets"] = measure_targets(args, rank, world, device)
         if not args.no_rows:
             res["rows"] = measure_rows(device)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             w = workload_from_args(args.workload, args.M, args.fmt)
-            v, unit, desc, threads = oracle_sample(w, budget_s=10.0)
-            res["cpu_baseline"] = {"value": v, "unit": unit, "cores": threads, "kind": "oracle",
-                                   "sample": desc}
+            r = oracle_sample(w, budget_s=8.0)
+            r1 = oracle_sample(w, budget_s=4.0, threads=1)
+            res["cpu_baseline"] = {"value": r["value"], "unit": r["unit"], "cores": r["threads"],
+                                   "kind": "oracle", "sample": r["sample"],
+                                   "single_core": {"value": r1["value"], "unit": r1["unit"], "cores": 1,
+                                                   "sample": r1["sample"]}}
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

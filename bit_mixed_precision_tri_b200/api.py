@@ -6,6 +6,7 @@ non-OK status and never fall back to another implementation.
 """
 from __future__ import annotations
 
+import collections
 import ctypes
 
 import torch
@@ -135,16 +136,28 @@ class Workspace:
         return self.buf
 
 
-_default_ws = {}
+_default_ws = collections.OrderedDict()
+_DEFAULT_WS_PER_DEVICE = 8
 
 
 def _workspace_for(device, stream_handle: int) -> Workspace:
     """The default workspace of (device, stream): calls on different streams
-    never share scratch, calls on one stream are ordered by it."""
-    key = (torch.device(device), int(stream_handle))
+    never share scratch, calls on one stream are ordered by it.  At most
+    ``_DEFAULT_WS_PER_DEVICE`` streams per device keep one (least recently
+    used dropped first), so short-lived streams do not pin device memory.  A
+    dropped buffer is released through the caching allocator, which keeps it
+    until the work already queued on its stream has used it (it was
+    allocated on that stream)."""
+    dev = torch.device(device)
+    key = (dev, int(stream_handle))
     ws = _default_ws.get(key)
     if ws is None:
-        ws = _default_ws[key] = Workspace(key[0])
+        ws = _default_ws[key] = Workspace(dev)
+        mine = [k for k in _default_ws if k[0] == dev]
+        for k in mine[:max(0, len(mine) - _DEFAULT_WS_PER_DEVICE)]:
+            del _default_ws[k]
+    else:
+        _default_ws.move_to_end(key)
     return ws
 
 

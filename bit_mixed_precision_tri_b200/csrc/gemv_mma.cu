@@ -542,29 +542,45 @@ cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const _
 // Static-scratch variant for callers that cannot allocate device memory.
 //
 // Some hosts of this library may not call cudaMalloc at all: a plugin inside
-// a framework that owns every device allocation, code that runs while a CUDA
-// graph is being captured (where an allocation would be recorded into, or
-// break, the capture), or a real-time loop that has to keep a fixed memory
-// footprint.  They still pass X, the packed weights and Y, but the scratch
-// this kernel needs (prepared activations, split-K partials, tickets) lives
-// in the file-scope array below instead of a caller-provided workspace.
+// a framework that owns every device allocation and hands out only the
+// tensors of the call, or a real-time or embedded loop that has to keep a
+// fixed, preallocated memory footprint.  They still pass X, the packed
+// weights and Y, but the scratch this kernel needs (prepared activations,
+// split-K partials, tickets) lives in the file-scope array below instead of
+// a caller-provided workspace.
 //
 // The array is a module global: every device that loads the library keeps
 // kNoAllocScratchBytes reserved until the process exits, and every call on a
 // device uses the same bytes, so calls that can overlap on that device (two
 // streams, or two host threads) race and must be ordered by the caller.
 // Host code only ever sees a host-side stand-in for the symbol; the device
-// address is looked up with cudaGetSymbolAddress once per device, with that
-// device current, on the first call there (which may also load the module, so
-// make that first call before any stream capture).
+// address is looked up with cudaGetSymbolAddress on the first call on each
+// device, with that device current (which may also load the module, so make
+// that first call before any stream capture).  A failed lookup is not
+// cached: the next call tries again.  What must start at zero (the per-tile
+// tickets) is cleared by the prep kernel of every call, inside the launch
+// sequence, so bytes left in the array by an earlier call never matter.
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
 constexpr int kMaxDev = 64;
 void* g_scratch_addr[kMaxDev];
-cudaError_t g_scratch_err[kMaxDev];
-std::once_flag g_scratch_once[kMaxDev];
+std::mutex g_scratch_mu[kMaxDev];
+
+// device address of the static array on the current device (looked up once
+// per device; only a successful lookup is kept)
+cudaError_t scratch_address(int dev, uint8_t** out) {
+  std::lock_guard<std::mutex> lock(g_scratch_mu[dev]);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = static_cast<uint8_t*>(g_scratch_addr[dev]);
+  return cudaSuccess;
+}
 }  // namespace
 
 size_t gemv_noalloc_scratch_limit() { return kNoAllocScratchBytes; }
@@ -579,17 +595,9 @@ cudaError_t launch_gemv_mma_noalloc(const __half* X, const uint8_t* qs, const __
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  std::call_once(g_scratch_once[dev], [dev]() {
-    void* ptr = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    g_scratch_addr[dev] = ptr;
-  });
-  if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
   if (gemv_noalloc_scratch_need(M, N, K, num_sms) > kNoAllocScratchBytes) return cudaErrorInvalidValue;
-  uint8_t* ws = static_cast<uint8_t*>(g_scratch_addr[dev]);
-  // the tickets (one per 128-row tile, at the head of the layout) must start
-  // at zero; the array keeps the last call's bytes
-  e = cudaMemsetAsync(ws, 0, up256((size_t)ceil_div(N, 128) * 4), s);
+  uint8_t* ws = nullptr;
+  e = scratch_address(dev, &ws);
   if (e != cudaSuccess) return e;
   return launch_gemv_mma(TRI_TQ2, X, qs, d, Y, M, N, K, ws, num_sms, s);
 }

@@ -212,18 +212,21 @@ TRI_API tri_status tri_gemm_tq1(const uint16_t* X, const uint8_t* qs, const uint
  * Ternary GEMM without any caller-provided workspace (TQ2, 1 <= M <= 16).
  * The pages have no counterpart: this is a deployment variant of the
  * decode-regime kernel for callers that may not allocate device memory (for
- * example a plugin whose host framework owns all allocations, or code that
- * runs while a CUDA graph is being captured).
+ * example a plugin whose host framework owns every device allocation and
+ * passes in only the call's tensors, or a real-time loop that must keep a
+ * fixed, preallocated memory footprint).
  *   Same result and argument meaning as tri_gemm_tq2 for these shapes; the
  *   scratch the kernel needs lives in a static 8 MiB device array inside the
  *   library, held on every device that loads it until the process exits.
  *   Returns TRI_ERR_SHAPE for M > 16 and TRI_ERR_SCRATCH_LIMIT when the shape
  *   needs more scratch than that array holds (tri_gemm_tq2_noalloc_fits
  *   answers beforehand).  It allocates nothing: the first call on a device
- *   looks the array up once for that device (and may load the module), so
- *   make that call before any stream capture.  All calls on a device share
- *   the array: calls that can run at the same time on that device (other
- *   streams, other host threads) race, so order them.
+ *   looks up the array's device address for that device (and may load the
+ *   module), so make that call before any stream capture; a lookup that
+ *   fails returns TRI_ERR_CUDA and is retried by the next call.  All calls
+ *   on a device share the array and each clears what it needs cleared:
+ *   calls that can run at the same time on that device (other streams,
+ *   other host threads) race, so order them.
  * ---------------------------------------------------------------------- */
 TRI_API tri_status tri_gemm_tq2_noalloc(const uint16_t* X, const uint8_t* qs, const uint16_t* d,
                                         uint16_t* Y, int64_t M, int64_t N, int64_t K,

@@ -62,19 +62,21 @@ def test_fused_block_layers():
 
 def test_oracle_sample_on_a_small_layer():
     w = dict(layers=[(256, 1024)], seeds=[0], M=1, fmt="tq2", name="tiny")
-    val, unit, desc, threads = bench.oracle_sample(w, budget_s=0.2)
-    assert unit == "GB/s" and val > 0 and threads >= 1 and "256x1024" in desc
+    r = bench.oracle_sample(w, budget_s=0.2)
+    assert r["unit"] == "GB/s" and r["value"] > 0 and r["threads"] >= 1 and "256x1024" in r["sample"]
+    assert r["elapsed_s"] >= 0.2
     w = dict(w, M=64)
-    val, unit, desc, threads = bench.oracle_sample(w, budget_s=0.2)
-    assert unit == "TFLOP/s" and val > 0
+    r = bench.oracle_sample(w, budget_s=0.2, threads=1)
+    assert r["unit"] == "TFLOP/s" and r["value"] > 0 and r["threads"] == 1
 
 
 def test_reference_arm_line(monkeypatch):
     calls = []
 
-    def fake_sample(w, budget_s=12.0):
+    def fake_sample(w, budget_s=12.0, threads=None):
         calls.append(budget_s)
-        return 0.025, "GB/s", "2 passes over the first min(N, 2048) rows of each layer", 16
+        return {"value": 0.025, "unit": "GB/s", "threads": 16, "elapsed_s": 2.5,
+                "sample": "2 passes over the first min(N, 2048) rows of each layer"}
 
     monkeypatch.setattr(bench, "oracle_sample", fake_sample)
     args = argparse.Namespace(workload="llama7b_decode_m1", M=None, fmt=None, steps=4, warmup=3)
@@ -85,9 +87,18 @@ def test_reference_arm_line(monkeypatch):
                 "cpu_baseline", "e2e"):
         assert key in line, key
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] == 0.025
+    assert line["ms_per_step"] == 2500.0                  # the measured time per step, not a budget
     assert line["config"]["workload"] == "llama7b_decode_m1" and line["dtype"] == "f64"
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] == 16 and cb["value"] == line["value"]
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert bench.run_reference(args, 1, 2) is None        # only rank 0 runs the oracle
+
+
+def test_default_workload_is_the_down_projection_decode():
+    src = open(bench.__file__).read()
+    assert 'ap.add_argument("--workload", default="down_8192x28672_m1"' in src
+    w = bench.WORKLOADS["down_8192x28672_m1"]
+    assert w["layers"] == [(8192, 28672)] and w["M"] == 1 and w["fmt"] == "tq2"
+    assert bench.TARGET_WORKLOADS == ("square_8192_m256", "llama7b_decode_m1")
