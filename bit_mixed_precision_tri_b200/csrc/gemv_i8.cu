@@ -33,13 +33,20 @@
 //    same number of weight bytes.  Each warp owns 16 rows of the tile and
 //    keeps four units of 16-byte cp.async copies in flight, the first four
 //    copied before the wait for the preceding grid.  A row tile split
-//    between CTAs is summed, in CTA order (deterministic), by the CTA that
-//    holds its first unit; the others leave partial sums stamped with the
-//    call's epoch (one 64-bit store each: no fence, no atomic).  The epoch is
-//    a counter on the device, one per workspace in a small library-owned
-//    pool, advanced by the last CTA of each call: bytes left in the
-//    workspace by earlier calls never pass for this call's sums, the
-//    workspace needs no clearing, and a captured graph replays correctly.
+//    between CTAs is finished by whichever CTA completes its share last:
+//    every contributing warp stores its rows' partial sums, stamped with the
+//    call (one 64-bit store each: no fence), and takes the warp's ticket of
+//    the tile (one atomic add); the warp that draws the last ticket adds the
+//    partials in CTA order (deterministic, whoever is last) and writes Y.  A
+//    value whose stamp is not yet this call's is one whose store was already
+//    issued (its warp took a ticket after it) and is read again until it
+//    lands: no CTA ever waits for work another CTA still has to do, so the
+//    result does not depend on which CTAs are resident together.  The stamp
+//    is a per-workspace call counter on the device (a small library-owned
+//    pool), advanced by the last CTA of each call, so bytes left in the
+//    workspace by earlier calls never pass for this call's sums; tickets live
+//    in the same pool, start at zero and are returned to zero by the warp
+//    that draws the last one.
 #include <mutex>
 
 #include "sm100_ptx.cuh"
@@ -47,9 +54,12 @@
 
 namespace tri {
 
-constexpr int kEpochSlots = 64;        // workspaces with an epoch slot per device
-// [slot][0]: epoch of the next call, [slot][1]: CTAs of the current call done
-static __device__ unsigned g_i8_epochs[kEpochSlots][2];
+constexpr int kEpochSlots = 32;        // workspaces with an epoch slot per device
+constexpr int kMaxG = 512;             // grid size limit
+// [slot][0]: epoch of the next call, [slot][1]: CTAs of the current call done,
+// [slot][2 + 8 c + w]: ticket of warp w for the row tile whose first CTA is c
+constexpr int kSlotWords = 2 + kMaxG * 8;
+static __device__ unsigned g_i8_epochs[kEpochSlots][kSlotWords];
 
 namespace {
 
@@ -60,8 +70,9 @@ constexpr float kQMax = 8.0e6f;        // |x^| bound: three balanced base-256 di
 
 struct Params {
   const __half* X;       // [M][K]
-  unsigned long long* partials;  // [G][kRT][M]: stamp << 32 | fp32 bits
-  unsigned* epoch;       // this workspace's [epoch, done] pair in the pool
+  unsigned long long* partials;  // [G][2][kRT][M]: stamp << 32 | fp32 bits; [c][0]: the CTA's last
+                                 // segment (a tile's start), [c][1]: its first (a tile continued)
+  unsigned* epoch;       // this workspace's [epoch, done, tickets...] words in the pool
   unsigned slot;         // its index (part of every stamp)
   unsigned* error;       // set when a wait for a partial sum gives up (never expected)
   int N, K, B, P, T, G;
@@ -337,24 +348,41 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
   int rt = (int)(u0 / P), q = q0;
   int seg_q0 = q, j = 0;
   const int r_local = warp * 16 + gid;
-  // Reducer of a split row tile: the CTA whose range holds the tile's first
-  // unit.  Every other CTA sharing the tile holds a prefix of its own range
-  // there (its first segment) or the whole range, so their partial sums come
-  // early; the bounded wait below normally finds them already written.
-  auto reduce_tile = [&](int tile) {
-    if (tig != 0) return;
-    const long long cfirst = blockIdx.x;
+  // End of a segment of row tile `tile` that does not cover the whole tile
+  // (side 0: it holds the tile's start, i.e. it is this CTA's last segment;
+  // side 1: it continues the tile, i.e. it is this CTA's first): store the
+  // warp's stamped partial sums, take the warp's ticket; the last arrival
+  // adds the partials of CTAs cfirst .. clast in order and writes Y.
+  auto finish_split = [&](int tile, int side) {
+    const long long cfirst = cta_of_unit((long long)tile * P, U, G);
     const long long clast = cta_of_unit((long long)tile * P + P - 1, U, G);
+    if (tig == 0) {
+      unsigned long long* mine = p.partials + ((size_t)blockIdx.x * 2 + side) * kRT * M;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+          __stcg(mine + (r_local + 8 * h) * M + m, (stamp << 32) | __float_as_uint(acc[h][m]));
+    }
+    __syncwarp();
+    unsigned old = 0;
+    unsigned* ticket = p.epoch + 2 + cfirst * kWarps + warp;
+    if (lane == 0) {
+      old = atomicAdd(ticket, 1u);
+      if (old == (unsigned)(clast - cfirst)) *ticket = 0u;   // nobody else touches it in this call
+    }
+    old = __shfl_sync(0xFFFFFFFFu, old, 0);
+    if (old != (unsigned)(clast - cfirst) || tig != 0) return;
     float sum[2][M];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int m = 0; m < M; ++m) sum[h][m] = acc[h][m];
+      for (int m = 0; m < M; ++m) sum[h][m] = 0.f;
     // The partial sums of up to kBatch contributors are loaded together (one
     // round trip), then checked and added in CTA order; only a value whose
-    // stamp is not yet this call's is polled again.
-    constexpr int kBatch = 8;
-    for (long long c0 = cfirst + 1; c0 <= clast; c0 += kBatch) {
+    // stamp is not yet this call's (a store still on its way) is read again.
+    constexpr int kBatch = 8 / M;
+    for (long long c0 = cfirst; c0 <= clast; c0 += kBatch) {
       const int nb = (int)(clast - c0 + 1 < kBatch ? clast - c0 + 1 : kBatch);
       unsigned long long v[kBatch][2][M];
 #pragma unroll
@@ -363,18 +391,26 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int m = 0; m < M; ++m)
-            v[k][h][m] = k < nb ? ptx::ld_relaxed_u64(p.partials + (size_t)(c0 + k) * kRT * M + (r_local + 8 * h) * M + m)
-                                : 0ull;
+            v[k][h][m] = (k < nb && c0 + k != (long long)blockIdx.x)
+                             ? ptx::ld_relaxed_u64(p.partials + ((size_t)(c0 + k) * 2 + (c0 + k == cfirst ? 0 : 1)) * kRT * M +
+                                                   (r_local + 8 * h) * M + m)
+                             : 0ull;
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {
         if (k >= nb) break;
+        const long long c = c0 + k;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int m = 0; m < M; ++m) {
+            if (c == (long long)blockIdx.x) {
+              sum[h][m] += acc[h][m];
+              continue;
+            }
             unsigned long long x = v[k][h][m];
-            const unsigned long long* a = p.partials + (size_t)(c0 + k) * kRT * M + (r_local + 8 * h) * M + m;
-            x = ptx::wait_stamp(a, x, stamp, kSpinLimit);
+            const unsigned long long* a =
+                p.partials + ((size_t)c * 2 + (c == cfirst ? 0 : 1)) * kRT * M + (r_local + 8 * h) * M + m;
+            x = ptx::wait_stamp(a, x, stamp, kSpinLimit);     // an issued store, bounded
             if ((x >> 32) != stamp) ptx::record_wait_failure(p.error, 11u);
             sum[h][m] += __uint_as_float((unsigned)x);
           }
@@ -470,23 +506,10 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
               for (int m = 0; m < M; ++m) Y[(size_t)m * p.N + n] = __float2half_rn(acc[h][m]);
           }
         }
-      } else if (u == n_units - 1 && seg_q0 == 0) {
-        // The segment holds the start of a row tile that continues in later
-        // CTAs: this CTA adds their partial sums (written when each finished
-        // its first segment, early in its range) after its own, in CTA order.
-        reduce_tile(cur_rt);
       } else {
-        // Any other split segment (the CTA's first, or its only one) ends in
-        // a partial sum stamped with the call's generation: one 64-bit store
-        // per value, no fence, no atomic.
-        if (tig == 0) {
-          unsigned long long* mine = p.partials + (size_t)blockIdx.x * kRT * M;
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int m = 0; m < M; ++m)
-              __stcg(mine + (r_local + 8 * h) * M + m, (stamp << 32) | __float_as_uint(acc[h][m]));
-        }
+        // a split segment: the tile's start (this CTA's last segment) or its
+        // continuation (this CTA's first)
+        finish_split(cur_rt, seg_q0 == 0 ? 0 : 1);
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -531,12 +554,13 @@ Layout layout_m(int64_t N, int64_t K, int num_sms) {
   if (G > per_sm * num_sms) G = per_sm * num_sms;
   if (G < 1) G = 1;
   if (ceil_div(L.U, G) > C::kMaxPairs) G = ceil_div(L.U, C::kMaxPairs);
+  if (G > kMaxG) G = kMaxG;
   L.G = (int)G;
   long long per = ceil_div(L.U, G);
   if (per > L.P) per = L.P;
   L.smem = (size_t)C::kRing + (size_t)per * C::kPairBytes;
   L.off_part = 0;
-  L.total = L.off_part + up256((size_t)G * kRT * M * 8);
+  L.total = L.off_part + up256((size_t)G * 2 * kRT * M * 8);
   return L;
 }
 
@@ -544,10 +568,16 @@ Layout layout_for(int64_t M, int64_t N, int64_t K, int num_sms) {
   return M == 1 ? layout_m<1>(N, K, num_sms) : layout_m<2>(N, K, num_sms);
 }
 
-// ---- epoch slots: one per (device, workspace); the least recently used is reused
+// ---- epoch slots: one per (device, workspace).  A slot's tickets are zero
+// between calls, so a slot may pass to another workspace once the calls of
+// its previous one are done: the slot reused is the least recently used one
+// last used on the calling stream (ordered with this call), else the least
+// recently used one.  (Calls in flight on other streams on more than
+// kEpochSlots workspaces at once could share a slot: not supported.)
 struct SlotTable {
   std::mutex mu;
   const void* ws[kEpochSlots] = {};
+  cudaStream_t stream[kEpochSlots] = {};
   unsigned long long used[kEpochSlots] = {};
   unsigned long long clock = 0;
   unsigned* base = nullptr;
@@ -555,7 +585,7 @@ struct SlotTable {
 constexpr int kMaxDev = 64;
 SlotTable g_slots[kMaxDev];
 
-cudaError_t epoch_slot(const void* ws, unsigned** out, unsigned* slot_out) {
+cudaError_t epoch_slot(const void* ws, cudaStream_t s, unsigned** out, unsigned* slot_out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -568,19 +598,21 @@ cudaError_t epoch_slot(const void* ws, unsigned** out, unsigned* slot_out) {
     if (e != cudaSuccess) return e;
     t.base = static_cast<unsigned*>(ptr);
   }
-  int slot = -1, lru = 0;
+  int slot = -1, lru = 0, lru_same = -1;
   for (int i = 0; i < kEpochSlots; ++i) {
     if (t.ws[i] == ws) { slot = i; break; }
     if (t.used[i] < t.used[lru]) lru = i;
+    if (t.stream[i] == s && (lru_same < 0 || t.used[i] < t.used[lru_same])) lru_same = i;
   }
   if (slot < 0) {
     // a reused slot keeps counting: stamps carry the slot index, so sums that
     // an earlier workspace left under another slot can never match
-    slot = lru;
+    slot = t.used[lru] == 0 ? lru : (lru_same >= 0 ? lru_same : lru);
     t.ws[slot] = ws;
   }
+  t.stream[slot] = s;
   t.used[slot] = ++t.clock;
-  *out = t.base + 2 * slot;
+  *out = t.base + (size_t)kSlotWords * slot;
   *slot_out = (unsigned)slot;
   return cudaSuccess;
 }
@@ -615,7 +647,7 @@ cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half
   Params p;
   p.X = X;
   p.partials = reinterpret_cast<unsigned long long*>(w + L.off_part);
-  cudaError_t e0 = epoch_slot(ws, &p.epoch, &p.slot);
+  cudaError_t e0 = epoch_slot(ws, s, &p.epoch, &p.slot);
   if (e0 != cudaSuccess) return e0;
   e0 = wait_status_word(&p.error);
   if (e0 != cudaSuccess) return e0;
@@ -639,7 +671,7 @@ cudaError_t launch_m(const __half* X, const uint8_t* qs, const __half* d, __half
 }  // namespace
 
 // Shapes whose per-CTA block pairs fit in shared memory with two CTAs per SM
-// (every CTA of the grid must be resident at once: reducers wait for others).
+// (within the grid size limit; no CTA waits for another, so any grid runs).
 bool gemv_i8_supported(int64_t M, int64_t N, int64_t K) {
   if (M >= 3) return gemv_i8n_supported(M, N, K);
   if (M < 1 || N < 1 || K < kBlock || K % kBlock) return false;
@@ -654,7 +686,9 @@ bool gemv_i8_supported(int64_t M, int64_t N, int64_t K) {
   const int sms = sm_count[dev];
   if (sms < 1) return false;
   const Layout L = layout_for(M, N, K, sms);
-  return L.G <= 2LL * sms;
+  long long per = ceil_div(L.U, L.G);
+  if (per > L.P) per = L.P;
+  return per <= (M == 1 ? Cfg<1>::kMaxPairs : Cfg<2>::kMaxPairs);
 }
 
 size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {

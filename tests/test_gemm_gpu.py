@@ -235,6 +235,65 @@ def test_i8_path_workspace_shared_with_other_paths():
         _check(Y8, X8, trits, d)
 
 
+@pytest.mark.parametrize("M", [1, 2])
+def test_i8_path_beside_a_concurrent_kernel(M):
+    """The decode kernel sums split row tiles through tickets (the last CTA to
+    finish a tile adds the partial sums), so no CTA waits for another: while
+    matrix products on a second stream hold a share of the SMs, the result is
+    still right."""
+    N, K = 8192, 7168
+    X, trits, qs, d = _case(M, N, K, 91 + M, "tq2")
+    Xd, qd, dd = torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV)
+    A = torch.randn(4096, 4096, dtype=torch.float16, device=DEV)
+    busy, mine = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    outs = []
+    with torch.cuda.stream(busy):
+        for _ in range(20):
+            A = (A @ A).clamp_(-1, 1)
+    with torch.cuda.stream(mine):
+        for _ in range(8):
+            outs.append(tri.gemm(Xd, qd, dd, N, K, "tq2", path=tri.PATH_I8, stream=mine))
+    torch.cuda.synchronize()
+    rows = np.arange(0, N, 7)
+    for Y in outs:
+        _check(Y[:, rows], X, trits[rows], d[rows])
+        assert torch.equal(Y, outs[0])
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_i8_path_chained_layers(M):
+    """Back-to-back decode GEMMs: the second reads the first one's output as
+    its activations (the kernel streams its weights before waiting for the
+    preceding grid, and reads X only after the wait)."""
+    K = 4096
+    trits1, g1 = O.absmean_ternarize(inputs.latent_weights(K, K, 85).numpy(), 1e-6)
+    trits2, g2 = O.absmean_ternarize(inputs.latent_weights(K, K, 86).numpy(), 1e-6)
+    q1, d1 = O.pack("tq2", trits1, np.array([g1], np.float32))
+    q2, d2 = O.pack("tq2", trits2, np.array([g2], np.float32))
+    X = inputs.activations(M, K, 87).numpy() * np.float16(0.05)
+    H = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(q1).to(DEV), torch.from_numpy(d1).to(DEV),
+                 K, K, "tq2", path=tri.PATH_I8)
+    Y = tri.gemm(H, torch.from_numpy(q2).to(DEV), torch.from_numpy(d2).to(DEV), K, K, "tq2",
+                 path=tri.PATH_I8)
+    Hh = H.cpu().numpy()
+    _check(H, X, trits1, d1)
+    _check(Y, Hh, trits2, d2)
+
+
+def test_i8_path_many_workspaces():
+    """More workspaces than the library keeps ticket rows for: rows pass from
+    one workspace to the next (their tickets are zero between calls)."""
+    M, N, K = 1, 1024, 4096
+    X, trits, qs, d = _case(M, N, K, 95, "tq2")
+    Xd, qd, dd = torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV)
+    wss = [tri.Workspace(DEV) for _ in range(300)]
+    outs = [tri.gemm(Xd, qd, dd, N, K, "tq2", path=tri.PATH_I8, workspace=w) for w in wss]
+    for Y in outs[::37] + outs[-2:]:
+        _check(Y, X, trits, d)
+    assert all(torch.equal(Y, outs[0]) for Y in outs)
+
+
 @pytest.mark.parametrize("M,N,K", [(17, 384, 512), (33, 256, 1024), (300, 520, 2304), (513, 384, 1280),
                                    (1024, 256, 768), (256, 1000, 11008), (129, 8192, 1024)])
 def test_tcgen05_path_shapes(M, N, K):
