@@ -60,10 +60,11 @@ WORKLOADS = {
 def kernels_per_call(path, M, fmt, swiglu=False):
     """Launches of this library's kernels for one call: prep + main for the
     mma.sync path and for the integer path at 3 <= M <= 16, one kernel
-    otherwise; TQ1 adds its transcode on the tensor-core paths; an unfused
+    otherwise; TQ1 adds its transcode on the tensor-core paths except the
+    integer path at M <= 2, which reads TQ1 planes directly; an unfused
     SwiGLU call adds its combine kernel."""
     n = 2 if path == 2 or (path == 4 and M >= 3) else 1
-    if fmt == "tq1" and path != 1:
+    if fmt == "tq1" and path != 1 and not (path == 4 and M <= 2):
         n += 1
     if swiglu and not (path == 4 and 3 <= M <= 16):
         n += 1

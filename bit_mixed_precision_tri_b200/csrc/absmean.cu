@@ -15,7 +15,8 @@
 // mean = RN64(S / (N*K)) and gamma = RN32(RN64(mean + eps)).
 //
 // Traffic: the bins pass reads W once (4 B/weight); ternarize reads W again
-// and writes one int8 per weight (5 B/weight).  Both are HBM-bound streams.
+// and writes one int8 per weight (5 B/weight).  Both are HBM-bound streams
+// with warp-contiguous accesses.
 #include "tri_internal.cuh"
 
 namespace tri {
@@ -161,27 +162,40 @@ __device__ __forceinline__ int8_t trit_of(float w, float g) {
   return (int8_t)__float2int_rn(x);
 }
 
+// Each thread handles four float4 of a 4 x kThreads-float4 chunk, at
+// stride kThreads, so every load and every 32-bit store of a warp is one
+// contiguous 512-byte (or 128-byte) run: W is read exactly once.
 __global__ void __launch_bounds__(kThreads)
 ternarize_kernel(const float* __restrict__ W, int64_t n, const float* __restrict__ gamma,
                  int8_t* __restrict__ trits) {
   const float g = *gamma;
-  const int64_t n16 = n >> 4;
-  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  const int64_t n4 = n >> 2;
+  const int64_t chunks = n4 / (4 * kThreads);
   const float4* W4 = reinterpret_cast<const float4*>(W);
-  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n16; i += stride) {
-    unsigned out[4];
+  unsigned* T4 = reinterpret_cast<unsigned*>(trits);
+  for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x) {
+    const int64_t base = c * 4 * kThreads + threadIdx.x;
+    float4 v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = ld_stream_f4(W4 + base + q * kThreads);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 v = ld_stream_f4(W4 + 4 * i + q);
-      const unsigned b0 = (unsigned)(uint8_t)trit_of(v.x, g);
-      const unsigned b1 = (unsigned)(uint8_t)trit_of(v.y, g);
-      const unsigned b2 = (unsigned)(uint8_t)trit_of(v.z, g);
-      const unsigned b3 = (unsigned)(uint8_t)trit_of(v.w, g);
-      out[q] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      const unsigned b0 = (unsigned)(uint8_t)trit_of(v[q].x, g);
+      const unsigned b1 = (unsigned)(uint8_t)trit_of(v[q].y, g);
+      const unsigned b2 = (unsigned)(uint8_t)trit_of(v[q].z, g);
+      const unsigned b3 = (unsigned)(uint8_t)trit_of(v[q].w, g);
+      T4[base + q * kThreads] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
     }
-    reinterpret_cast<uint4*>(trits)[i] = make_uint4(out[0], out[1], out[2], out[3]);
   }
-  for (int64_t i = (n16 << 4) + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride)
+  // the float4 after the last whole chunk, then single elements
+  for (int64_t i = chunks * 4 * kThreads + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * kThreads) {
+    const float4 v = ld_stream_f4(W4 + i);
+    T4[i] = (unsigned)(uint8_t)trit_of(v.x, g) | ((unsigned)(uint8_t)trit_of(v.y, g) << 8) |
+            ((unsigned)(uint8_t)trit_of(v.z, g) << 16) | ((unsigned)(uint8_t)trit_of(v.w, g) << 24);
+  }
+  for (int64_t i = (n4 << 2) + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * kThreads)
     trits[i] = trit_of(W[i], g);
 }
 
@@ -212,7 +226,7 @@ cudaError_t launch_absmean(const float* W, int64_t n, float eps, float* gamma, v
 
 cudaError_t launch_ternarize(const float* W, int64_t n, const float* gamma, int8_t* trits,
                              cudaStream_t s) {
-  ternarize_kernel<<<grid_for(n >> 4), kThreads, 0, s>>>(W, n, gamma, trits);
+  ternarize_kernel<<<grid_for(n >> 4), kThreads, 0, s>>>(W, n, gamma, trits);   // one block per 4 x 256 float4
   return cudaGetLastError();
 }
 

@@ -44,28 +44,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// As mbar_try_wait, with a hint (in ns) for how long the hardware may keep
-// the thread suspended waiting for the phase: a waiting warp then takes no
-// issue slots from the warps that do the work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
-  return ok != 0;
-}
-
-// Bounded wait with a suspend hint per poll; returns false after `limit`
-// polls, never spins forever.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t limit,
-                                                uint32_t hint_ns) {
-  for (uint32_t i = 0; i < limit; ++i)
-    if (mbar_try_wait_sleep(bar, parity, hint_ns)) return true;
-  return false;
-}
-
 // Bounded wait: returns false after `limit` polls (each poll is a hardware
 // try_wait that itself suspends for a while), never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
@@ -220,9 +198,10 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ordered after the surrounding synchronisation (memory clobber)
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {

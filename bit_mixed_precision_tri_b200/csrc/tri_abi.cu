@@ -59,29 +59,34 @@ tri_status check_nk(int64_t N, int64_t K) {
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// The tensor-core kernels consume TQ2 planes; TQ1 weights reach them through
-// a transcode into the head of the workspace (N*K/4 bytes).
+// The integer path reads TQ1 planes directly for M <= 2 (the decode
+// regime, where the weight stream is the cost); the other tensor-core kernels
+// consume TQ2 planes, and TQ1 weights reach them through a transcode into the
+// head of the workspace (N*K/4 bytes).
+bool tq1_direct(int fmt, int path, int64_t M) { return fmt == TRI_TQ1 && path == TRI_PATH_I8 && M <= 2; }
+
 bool path_supported(int fmt, int path, int64_t M, int64_t N, int64_t K) {
-  (void)fmt;
   switch (path) {
     case TRI_PATH_SIMT: return true;
     case TRI_PATH_MMA: return tri::gemv_mma_supported(TRI_TQ2, M, N, K);
     case TRI_PATH_TCGEN05: return tri::gemm_tc_supported(TRI_TQ2, M, N, K);
-    case TRI_PATH_I8: return tri::gemv_i8_supported(M, N, K);
+    case TRI_PATH_I8: return tri::gemv_i8_supported(M, N, K, tq1_direct(fmt, path, M));
     default: return false;
   }
 }
 
-size_t transcode_bytes(int fmt, int path, int64_t N, int64_t K) {
-  return (fmt == TRI_TQ1 && path != TRI_PATH_SIMT) ? up256((size_t)N * (size_t)K / 4) : 0;
+size_t transcode_bytes(int fmt, int path, int64_t M, int64_t N, int64_t K) {
+  return (fmt == TRI_TQ1 && path != TRI_PATH_SIMT && !tq1_direct(fmt, path, M))
+             ? up256((size_t)N * (size_t)K / 4)
+             : 0;
 }
 
 size_t path_ws_bytes(int fmt, int path, int64_t M, int64_t N, int64_t K, int sms) {
   size_t inner = 0;
   if (path == TRI_PATH_MMA) inner = tri::gemv_mma_ws_bytes(TRI_TQ2, M, N, K, sms);
   if (path == TRI_PATH_TCGEN05) inner = tri::gemm_tc_ws_bytes(TRI_TQ2, M, N, K, sms);
-  if (path == TRI_PATH_I8) inner = tri::gemv_i8_ws_bytes(M, N, K, sms);
-  return transcode_bytes(fmt, path, N, K) + inner;
+  if (path == TRI_PATH_I8) inner = tri::gemv_i8_ws_bytes(M, N, K, sms, tq1_direct(fmt, path, M));
+  return transcode_bytes(fmt, path, M, N, K) + inner;
 }
 
 int auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
@@ -232,19 +237,21 @@ tri_status tri_gemm(int format, int path, const uint16_t* X, const uint8_t* qs, 
   if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
   const uint8_t* q2 = qs;
   uint8_t* inner = static_cast<uint8_t*>(workspace);
-  if (format == TRI_TQ1) {
+  const bool direct = tq1_direct(format, path, M);
+  if (format == TRI_TQ1 && !direct) {
     uint8_t* t = static_cast<uint8_t*>(workspace);
     const cudaError_t e = tri::launch_transcode_tq1_tq2(qs, N, K, t, s);
     if (e != cudaSuccess) return from_cuda(e);
     q2 = t;
-    inner = t + transcode_bytes(format, path, N, K);
+    inner = t + transcode_bytes(format, path, M, N, K);
   }
   switch (path) {
     case TRI_PATH_MMA:
       return from_cuda(tri::launch_gemv_mma(TRI_TQ2, Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner,
                                             di.sms, s));
     case TRI_PATH_I8:
-      return from_cuda(tri::launch_gemv_i8(Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner, di.sms, s));
+      return from_cuda(
+          tri::launch_gemv_i8(Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner, di.sms, s, direct));
     case TRI_PATH_TCGEN05:
       return from_cuda(tri::launch_gemm_tc(TRI_TQ2, Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner,
                                            di.sms, s));
@@ -293,12 +300,13 @@ tri_status tri_gemm_swiglu(int format, int path, const uint16_t* X, const uint8_
   if (workspace && !aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
   const uint8_t* q2 = qs;
   uint8_t* inner = static_cast<uint8_t*>(workspace);
-  if (format == TRI_TQ1 && path != TRI_PATH_SIMT) {
+  const bool direct = tq1_direct(format, path, M);
+  if (format == TRI_TQ1 && path != TRI_PATH_SIMT && !direct) {
     uint8_t* t = static_cast<uint8_t*>(workspace);
     const cudaError_t e = tri::launch_transcode_tq1_tq2(qs, N, K, t, s);
     if (e != cudaSuccess) return from_cuda(e);
     q2 = t;
-    inner = t + transcode_bytes(format, path, N, K);
+    inner = t + transcode_bytes(format, path, M, N, K);
   }
   if (fused)
     return from_cuda(tri::launch_gemv_i8n(Xh, q2, dh, Yh, (int)M, (int)N, (int)K, inner, di.sms, s, true));
@@ -313,7 +321,7 @@ tri_status tri_gemm_swiglu(int format, int path, const uint16_t* X, const uint8_
       e = tri::launch_gemv_mma(TRI_TQ2, Xh, q2, dh, G2, (int)M, (int)N, (int)K, inner, di.sms, s);
       break;
     case TRI_PATH_I8:
-      e = tri::launch_gemv_i8(Xh, q2, dh, G2, (int)M, (int)N, (int)K, inner, di.sms, s);
+      e = tri::launch_gemv_i8(Xh, q2, dh, G2, (int)M, (int)N, (int)K, inner, di.sms, s, direct);
       break;
     case TRI_PATH_TCGEN05:
       e = tri::launch_gemm_tc(TRI_TQ2, Xh, q2, dh, G2, (int)M, (int)N, (int)K, inner, di.sms, s);

@@ -49,8 +49,8 @@ cudaError_t launch_gemv_mma(int fmt, const __half* X, const uint8_t* qs, const _
                             __half* Y, int M, int N, int K, void* ws, int num_sms,
                             cudaStream_t s);
 
-// decode-regime integer tensor-core path (TQ2, M <= 16: gemv_i8.cu for M <= 2,
-// gemv_i8n.cu for 3 <= M <= 16)
+// decode-regime integer tensor-core path (M <= 16: gemv_i8.cu for M <= 2, TQ2
+// or TQ1 planes read directly; gemv_i8n.cu for 3 <= M <= 16, TQ2)
 bool gemv_i8n_supported(int64_t M, int64_t N, int64_t K);
 size_t gemv_i8n_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 // swiglu: N = 2F rows of gate and up interleaved in groups of 8, Y = silu(gate) * up [M][F]
@@ -58,10 +58,11 @@ cudaError_t launch_gemv_i8n(const __half* X, const uint8_t* qs, const __half* d,
                             int K, void* ws, int num_sms, cudaStream_t s, bool swiglu = false);
 // silu(G) * U from a [M][2F] fp16 product in the interleaved row order, into Y [M][F]
 cudaError_t launch_swiglu_combine(const __half* G2, __half* Y, int64_t M, int64_t F, cudaStream_t s);
-bool gemv_i8_supported(int64_t M, int64_t N, int64_t K);
-size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+// tq1: qs is a TQ1 plane (M <= 2 only)
+bool gemv_i8_supported(int64_t M, int64_t N, int64_t K, bool tq1 = false);
+size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms, bool tq1 = false);
 cudaError_t launch_gemv_i8(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M,
-                           int N, int K, void* ws, int num_sms, cudaStream_t s);
+                           int N, int K, void* ws, int num_sms, cudaStream_t s, bool tq1 = false);
 
 // decode-regime path with library-owned static scratch (no allocation)
 size_t gemv_noalloc_scratch_limit();

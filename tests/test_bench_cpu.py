@@ -31,7 +31,9 @@ def test_decode_set_weight_bytes_per_layer():
     (PATH_I8, 2, "tq2", False, 1),
     (PATH_I8, 3, "tq2", False, 2),        # 3 <= M <= 16: prep + main
     (PATH_I8, 16, "tq2", False, 2),
-    (PATH_I8, 1, "tq1", False, 2),        # TQ1: + the TQ1 -> TQ2 transcode
+    (PATH_I8, 1, "tq1", False, 1),        # M <= 2 reads TQ1 planes directly
+    (PATH_I8, 2, "tq1", True, 2),         # + the SwiGLU combine
+    (PATH_I8, 4, "tq1", False, 3),        # 3 <= M <= 16: + the TQ1 -> TQ2 transcode
     (PATH_I8, 8, "tq2", True, 2),         # SwiGLU fused into the integer kernel's epilogue
     (PATH_I8, 2, "tq2", True, 2),         # ... but not for M <= 2: + the combine kernel
     (PATH_MMA, 4, "tq2", False, 2),       # prep + main

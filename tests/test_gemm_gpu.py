@@ -167,13 +167,14 @@ def test_i8_path_shapes(fmt, M, N, K):
     _check(Y, X, trits, d)
 
 
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
 @pytest.mark.parametrize("M", [1, 2])
-def test_i8_path_activation_extremes(M):
+def test_i8_path_activation_extremes(M, fmt):
     """Fixed-point activations: a block holding one value near the fp16 maximum
     among tiny ones (the quantisation step is set by the largest |x| of the
     block), an all-zero block, subnormal values and signed extremes."""
     N, K = 384, 2048
-    X, trits, qs, d = _case(M, N, K, 41, "tq2", per_block=True, p_zero=0.5)
+    X, trits, qs, d = _case(M, N, K, 41, fmt, per_block=True, p_zero=0.5)
     X = X.copy()
     X[:, 0] = 60000.0
     X[:, 1:256] = (np.random.default_rng(3).standard_normal((M, 255)) * 1e-3).astype(np.float16)
@@ -182,8 +183,46 @@ def test_i8_path_activation_extremes(M):
     X[:, 768] = -65504.0
     X[:, 769] = 65504.0
     Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
-                 torch.from_numpy(d).to(DEV), N, K, "tq2", path=tri.PATH_I8)
+                 torch.from_numpy(d).to(DEV), N, K, fmt, path=tri.PATH_I8)
     _check(Y, X, trits, d)
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_i8_path_tq1_any_byte(M):
+    """TQ1 planes read directly at M <= 2: every byte value, the ones no packer
+    writes included, decodes as the inverse formula does (N5 = floor(243 b /
+    256), digits first-most-significant; the last byte of a block gives one
+    trit), so the product matches the oracle's product of its decoded trits."""
+    N, K = 640, 2816
+    rng = np.random.default_rng(55 + M)
+    qs = rng.integers(0, 256, size=(N, (K // 256) * 52), dtype=np.uint8)
+    for r in range(4):                    # every byte value in every position of a row
+        qs[r] = np.resize(np.roll(np.arange(256, dtype=np.uint8), 64 * r), qs.shape[1])
+    trits, invalid = O.unpack_tq1(qs, N, K)
+    assert invalid > 0
+    d = O.block_scales_fp16(rng.uniform(0.005, 0.05, size=N * (K // 256)).astype(np.float32), N, K)
+    X = inputs.activations(M, K, 56).numpy()
+    Y = tri.gemm(torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV),
+                 torch.from_numpy(d).to(DEV), N, K, "tq1", path=tri.PATH_I8)
+    _check(Y, X, trits, d)
+
+
+@pytest.mark.parametrize("M", [1, 2])
+def test_i8_path_tq1_plane_4_byte_aligned(M):
+    """A TQ1 plane that starts 4 bytes past a 16-byte boundary (the format
+    only needs 4): the rows are then copied word by word instead of in
+    16-byte chunks, with the same result."""
+    N, K = 300, 4096
+    X, trits, qs, d = _case(M, N, K, 61 + M, "tq1", per_block=True, p_zero=0.31)
+    buf = torch.zeros(qs.size + 16, dtype=torch.uint8, device=DEV)
+    shifted = buf[4:4 + qs.size].view(qs.shape)
+    shifted.copy_(torch.from_numpy(qs).to(DEV))
+    assert shifted.data_ptr() % 16 == 4
+    Xd, dd = torch.from_numpy(X).to(DEV), torch.from_numpy(d).to(DEV)
+    Y = tri.gemm(Xd, shifted, dd, N, K, "tq1", path=tri.PATH_I8)
+    _check(Y, X, trits, d)
+    Y16 = tri.gemm(Xd, torch.from_numpy(qs).to(DEV), dd, N, K, "tq1", path=tri.PATH_I8)
+    assert torch.equal(Y, Y16)
 
 
 def test_i8_path_deterministic():
