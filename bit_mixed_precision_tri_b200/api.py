@@ -161,10 +161,35 @@ def _workspace_for(device, stream_handle: int) -> Workspace:
     return ws
 
 
+class WaitGaveUp(RuntimeError):
+    """A bounded wait inside a GEMM kernel ran out (code in ``.code``); the
+    output of the call is unspecified."""
+
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: a bounded wait in the kernel gave up (code {code})")
+
+
+def _check_waits(device, stream_handle: int, what: str) -> None:
+    """Synchronize `stream_handle`, read and clear the device's wait status
+    word, raise WaitGaveUp when a wait gave up."""
+    code = ctypes.c_uint32(0)
+    with torch.cuda.device(device):
+        st = _lib.lib().tri_wait_status(ctypes.byref(code), 1, stream_handle)
+    if st:
+        _lib.check(st, "tri_wait_status")
+    if code.value:
+        raise WaitGaveUp(int(code.value), what)
+
+
 def gemm(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, N: int, K: int, fmt="tq2",
          path: int = PATH_AUTO, out: torch.Tensor = None, workspace: Workspace = None,
-         stream=None) -> torch.Tensor:
-    """Y = X (d * W_hat)^T in fp16 with fp32 accumulation."""
+         stream=None, check: bool = False) -> torch.Tensor:
+    """Y = X (d * W_hat)^T in fp16 with fp32 accumulation.
+
+    ``check=True`` (for debugging; it synchronizes the stream) reads the
+    device's wait status word after the call and raises WaitGaveUp if a
+    bounded wait inside the kernel ran out."""
     # the checks a decode step pays on every call, kept to attribute reads
     if not (X.is_cuda and qs.is_cuda and d.is_cuda):
         raise ValueError("tensors must live on a CUDA device")
@@ -186,6 +211,8 @@ def gemm(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, N: int, K: int, fmt
                              M, N, K, ws.data_ptr(), ws.numel(), s)
     if st:
         _lib.check(st, "tri_gemm")
+    if check:
+        _check_waits(X.device, s, "tri_gemm")
     return Y
 
 
@@ -209,9 +236,9 @@ def interleave_gate_up(qs_gate: torch.Tensor, d_gate: torch.Tensor, qs_up: torch
 
 def gemm_swiglu(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, F: int, K: int, fmt="tq2",
                 path: int = PATH_AUTO, out: torch.Tensor = None, workspace: Workspace = None,
-                stream=None) -> torch.Tensor:
+                stream=None, check: bool = False) -> torch.Tensor:
     """Y = silu(X Wg^T) * (X Wu^T), fp16 [M][F], from the interleaved 2F-row
-    packed weights of ``interleave_gate_up``."""
+    packed weights of ``interleave_gate_up``; ``check`` as in ``gemm``."""
     if not (X.is_cuda and qs.is_cuda and d.is_cuda):
         raise ValueError("tensors must live on a CUDA device")
     if not (X.is_contiguous() and qs.is_contiguous() and d.is_contiguous()):
@@ -234,6 +261,8 @@ def gemm_swiglu(X: torch.Tensor, qs: torch.Tensor, d: torch.Tensor, F: int, K: i
                            M, F, K, ws.data_ptr(), ws.numel(), s)
     if st:
         _lib.check(st, "tri_gemm_swiglu")
+    if check:
+        _check_waits(X.device, s, "tri_gemm_swiglu")
     return Y
 
 

@@ -382,6 +382,21 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
     const int f_tig = f_word >> 2, f_p = (f_word >> 1) & 1, f_r = f_word & 1;
     constexpr int kXB = 4;
     const int n_blk = n_pairs * 2;
+    // TQ1: this lane's eight slots (prefix registers 2 (L % 8) + r of lane
+    // tig = L / 8, bytes bi): the index k0 of x_j, whether x_{j+1} enters
+    // (j < 5 inside the block), and the record offset of the words
+    int tq_k0[8];
+    uint32_t tq_two = 0;
+    const int tq_rec = (((lane & 7) >> 1) * C::kBSlots + (lane >> 3)) * 16 + (lane & 1) * 8;
+    if constexpr (kTQ1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        int g, jp;
+        tq1_slot(lane >> 3, 2 * (lane & 7) + (e >> 2), e & 3, g, jp);
+        tq_k0[e] = 5 * g + jp - 1;
+        if (jp < 5 && tq_k0[e] + 1 < kBlock) tq_two |= 1u << e;
+      }
+    }
     for (int hb0 = warp; hb0 < n_blk; hb0 += kXB * kWarps) {
       uint4 raw[kXB][M];
 #pragma unroll
@@ -448,27 +463,22 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
             reinterpret_cast<int4*>(xs)[2 * lane] = make_int4(qv[0], qv[1], qv[2], qv[3]);
             reinterpret_cast<int4*>(xs)[2 * lane + 1] = make_int4(qv[4], qv[5], qv[6], qv[7]);
             __syncwarp();
-            const int tk = lane >> 3, mi = lane & 7;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
               uint32_t dg[4];
 #pragma unroll
               for (int bi = 0; bi < 4; ++bi) {
-                int g, jp;
-                tq1_slot(tk, 2 * mi + r, bi, g, jp);
-                const int k0 = 5 * g + jp - 1;
-                const int a = xs[k0];
-                const int b = (jp < 5 && k0 + 1 < kBlock) ? xs[k0 + 1] : 0;
-                const int v = jp < 5 ? a - 3 * b : a;
-                dg[bi] = ((uint32_t)v + 0x80808080u) ^ 0x80808080u;
+                const int e = 4 * r + bi;
+                const int a = xs[tq_k0[e]];
+                const int b = (tq_two >> e) & 1u ? xs[tq_k0[e] + 1] : 0;
+                dg[bi] = ((uint32_t)(a - 3 * b) + 0x80808080u) ^ 0x80808080u;
               }
 #pragma unroll
               for (int lv = 0; lv < 4; ++lv) {
                 const uint32_t sel = (uint32_t)(3 - lv) | ((uint32_t)(7 - lv) << 4);
                 const uint32_t lo = __byte_perm(dg[0], dg[1], sel), hi = __byte_perm(dg[2], dg[3], sel);
                 const uint32_t word = (lo & 0xFFFFu) | (hi << 16);
-                *reinterpret_cast<uint32_t*>(rec + (((mi >> 1) * C::kBSlots + (4 * m + lv) * 4 + tk) * 16 +
-                                                    (mi & 1) * 8 + r * 4)) = word;
+                *reinterpret_cast<uint32_t*>(rec + tq_rec + (4 * m + lv) * 4 * 16 + r * 4) = word;
               }
             }
             __syncwarp();                             // the staging row is free for the next block

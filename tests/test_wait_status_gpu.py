@@ -75,3 +75,27 @@ def test_healthy_calls_leave_status_zero(M, path):
         Y = tri.gemm(Xd, qs_t, d_t, N, K, "tq2", path=path)
     assert tri.wait_status(DEV) == 0
     _assert_close(Y, X, trits, d)
+
+
+@pytest.mark.parametrize("fmt", ["tq2", "tq1"])
+def test_gemm_check_option(fmt):
+    """gemm(check=True) returns normally after healthy calls, and raises
+    WaitGaveUp when the word holds a code (here one left by the self-test
+    kernel just before the call), clearing it."""
+    tri.wait_status(DEV, clear=True)
+    M, N, K = 1, 1024, 4096
+    W = inputs.latent_weights(N, K, 3)
+    trits, g = O.absmean_ternarize(W.numpy(), 1e-6)
+    qs, d = O.pack(fmt, trits, np.array([g], np.float32))
+    X = inputs.activations(M, K, 4).numpy()
+    args = (torch.from_numpy(X).to(DEV), torch.from_numpy(qs).to(DEV), torch.from_numpy(d).to(DEV), N, K, fmt)
+    Y = tri.gemm(*args, check=True)
+    _assert_close(Y, X, trits, d)
+    tri.selftest_wait_timeout(1, DEV)
+    with pytest.raises(tri.WaitGaveUp) as e:
+        tri.gemm(*args, check=True)
+    assert e.value.code == 91
+    assert tri.wait_status(DEV) == 0
+    Y = tri.gemm_swiglu(torch.from_numpy(np.ascontiguousarray(X)).to(DEV), *tri.interleave_gate_up(
+        args[1][:512], args[2][:512], args[1][512:], args[2][512:]), 512, K, fmt, check=True)
+    assert Y.shape == (M, 512)
