@@ -639,6 +639,9 @@ def main():
                     help="skip the extra target workloads of the default line")
     ap.add_argument("--sweep", action="store_true",
                     help="print one line per batch-sweep, block and format-stress workload")
+    ap.add_argument("--rows-only", action="store_true",
+                    help="time only the offline rows (absmean, ternarize, pack, unpack) on the "
+                         "28672x8192 weight, --steps timed calls each, and print them")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -661,6 +664,10 @@ def main():
     try:
         if args.sweep:
             run_sweep(args, rank, world, device)
+            return
+        if args.rows_only:
+            if rank == 0:
+                print(json.dumps({"rows": measure_rows(device, reps=max(1, args.steps))}), flush=True)
             return
         res = run_ours(args, rank, world, device)
         if not args.no_cublas:

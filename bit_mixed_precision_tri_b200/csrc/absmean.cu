@@ -7,12 +7,22 @@
 //
 // Exactness.  A trit flips if gamma moves by one ulp near |W/gamma| = 0.5, so
 // gamma must not depend on the reduction order.  Every finite float32 |w| is
-// m * 2^(e-150) with a 24-bit integer m and e = max(biased exponent, 1); the
-// kernel sums the integers m per exponent e into 64-bit bins (integer adds
-// commute, so the bins are identical for every grid and every run), and a
-// one-thread finalize expands sum_e bin[e] * 2^(e-1) into a 352-bit integer
-// (units of 2^-149) and rounds it once to the nearest double.  Then
-// mean = RN64(S / (N*K)) and gamma = RN32(RN64(mean + eps)).
+// m * 2^(e-150) with a 24-bit integer m and e = max(biased exponent, 1), i.e.
+// m * 2^(e-1) in units of 2^-149.  All sums are of such integers (integer adds
+// commute, so the result is identical for every grid and every run): a bin
+// b holds integers worth 2^(b-1) units each, and a one-thread finalize
+// expands sum_b bin[b] * 2^(b-1) into a 384-bit integer and rounds it once to
+// the nearest double.  Then mean = RN64(S / (N*K)) and gamma =
+// RN32(RN64(mean + eps)).
+//
+// The bins pass keeps, per lane, a window of 24 exponents [lo, lo + 23]
+// placed below the largest exponent the lane has seen: the lane adds
+// m << (e - lo) (< 2^47) into a 64-bit register, which is flushed as two
+// 32-bit halves into the warp's shared bins lo and lo + 32 when the window
+// moves up, every 2^16 values and at the end.  A value below the window (for
+// real weights, below 2^-22 of the lane's largest magnitude: rare) is added
+// to its own bin at once (one shared atomic).  No warp collective runs in the
+// loop.
 //
 // Traffic: the bins pass reads W once (4 B/weight); ternarize reads W again
 // and writes one int8 per weight (5 B/weight).  Both are HBM-bound streams
@@ -22,7 +32,7 @@
 namespace tri {
 namespace {
 
-constexpr int kBins = 256;
+constexpr int kBins = 288;          // exponents 1..254, and flushed high halves up to 254 + 10
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
@@ -39,22 +49,64 @@ __device__ __forceinline__ float4 ld_stream_f4(const float4* p) {
   return v;
 }
 
-// Add |x| to the warp's exponent bins.  Lanes holding the same exponent are
-// grouped with match.any, their 24-bit mantissas summed with redux.sync
-// (< 2^29, exact in 32 bits), and one lane per group issues the atomic, so a
-// warp step costs one shared atomic per distinct exponent instead of 32.
-// All 32 lanes must call this together.
-__device__ __forceinline__ void bin_add_warp(unsigned long long* wbins, float x, unsigned& bad) {
-  const unsigned u = __float_as_uint(x) & 0x7FFFFFFFu;
-  unsigned e = u >> 23;
-  unsigned m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-  if (e == 255u) { bad = 1u; m = 0u; }
-  if (e == 0u) e = 1u;
-  const unsigned grp = __match_any_sync(0xFFFFFFFFu, e);
-  const unsigned sum = __reduce_add_sync(grp, m);
-  if ((threadIdx.x & 31) == (unsigned)(__ffs(grp) - 1) && sum != 0u)
-    atomicAdd(&wbins[e], (unsigned long long)sum);
-}
+// One lane's window accumulator: exponents lo .. lo + 23 (placed below the
+// largest exponent the lane has seen), acc = sum of m << (e - lo) < 2^63
+// (at most 2^16 values of < 2^47 between flushes).  A flush adds the two
+// 32-bit halves to bins lo and lo + 32; a value below the window goes to its
+// own bin at once (rare for real weights: below 2^-22 of the lane's largest).
+struct LaneAcc {
+  int lo = 0;                    // 0: no window yet
+  int cnt = 0;                   // values added since the last flush
+  unsigned long long acc = 0ull;
+
+  __device__ __forceinline__ void flush(unsigned long long* wb) {
+    if (acc) {
+      atomicAdd(&wb[lo], acc & 0xFFFFFFFFull);
+      if (acc >> 32) atomicAdd(&wb[lo + 32], acc >> 32);
+    }
+    acc = 0ull;
+    cnt = 0;
+  }
+
+  template <int K>
+  __device__ __forceinline__ void add(unsigned long long* wb, const float (&x)[K], unsigned& bad) {
+    unsigned e[K], m[K];
+    unsigned emax = 1u;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      // e = max(biased exponent, 1); m = fraction plus the hidden bit
+      // exactly when the biased exponent is not 0 (zero and denormals)
+      const unsigned bits = __float_as_uint(x[i]);
+      const unsigned er = (bits >> 23) & 0xFFu;
+      e[i] = er > 1u ? er : 1u;
+      m[i] = (bits & 0x7FFFFFu) + 0x800000u - ((e[i] - er) << 23);
+      emax = e[i] > emax ? e[i] : emax;
+    }
+    if (emax == 255u) {          // Inf or NaN somewhere: gamma becomes NaN (rare)
+      bad = 1u;
+      emax = 1u;
+#pragma unroll
+      for (int i = 0; i < K; ++i) {
+        if (e[i] == 255u) {
+          m[i] = 0u;
+          e[i] = 1u;
+        }
+        emax = e[i] > emax ? e[i] : emax;
+      }
+    }
+    if (lo == 0 || (int)emax > lo + 23 || cnt > (1 << 16) - K) {
+      flush(wb);
+      lo = (int)emax - 22 > 1 ? (int)emax - 22 : 1;
+    }
+    cnt += K;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+      const int dsh = (int)e[i] - lo;
+      if (dsh >= 0) acc += (unsigned long long)m[i] << dsh;
+      else if (m[i]) atomicAdd(&wb[e[i]], (unsigned long long)m[i]);
+    }
+  }
+};
 
 __global__ void __launch_bounds__(kThreads)
 absmean_bins_kernel(const float* __restrict__ W, int64_t n, AbsmeanWs* ws) {
@@ -66,20 +118,39 @@ absmean_bins_kernel(const float* __restrict__ W, int64_t n, AbsmeanWs* ws) {
   const int64_t n4 = n >> 2;
   const float4* W4 = reinterpret_cast<const float4*>(W);
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  // whole warps iterate together (the bins update is a warp collective)
-  for (int64_t base = (int64_t)blockIdx.x * kThreads; base < n4; base += stride) {
-    const int64_t i = base + threadIdx.x;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < n4) v = ld_stream_f4(W4 + i);
-    bin_add_warp(wb, v.x, bad);
-    bin_add_warp(wb, v.y, bad);
-    bin_add_warp(wb, v.z, bad);
-    bin_add_warp(wb, v.w, bad);
+  LaneAcc la;
+  // Chunks of 4 x kThreads float4: every thread has four 16-byte loads in
+  // flight, each warp-wide load one contiguous 512 bytes.
+  // The next chunk's loads are issued before the current one is added up.
+  const int64_t chunks = n4 / (4 * kThreads);
+  float4 v[4];
+  if ((int64_t)blockIdx.x < chunks) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = ld_stream_f4(W4 + (int64_t)blockIdx.x * 4 * kThreads + threadIdx.x + q * kThreads);
   }
-  for (int64_t base = (n4 << 2) + (int64_t)blockIdx.x * kThreads; base < n; base += stride) {
-    const int64_t i = base + threadIdx.x;
-    bin_add_warp(wb, i < n ? W[i] : 0.f, bad);
+  for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x) {
+    const int64_t cn = c + gridDim.x;
+    float4 w[4];
+    if (cn < chunks) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[q] = ld_stream_f4(W4 + cn * 4 * kThreads + threadIdx.x + q * kThreads);
+    }
+    const float x[16] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w,
+                         v[2].x, v[2].y, v[2].z, v[2].w, v[3].x, v[3].y, v[3].z, v[3].w};
+    la.add<16>(wb, x, bad);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = w[q];
   }
+  for (int64_t i = chunks * 4 * kThreads + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n4; i += stride) {
+    const float4 v = ld_stream_f4(W4 + i);
+    const float x[4] = {v.x, v.y, v.z, v.w};
+    la.add<4>(wb, x, bad);
+  }
+  for (int64_t i = (n4 << 2) + (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n; i += stride) {
+    const float x[1] = {W[i]};
+    la.add<1>(wb, x, bad);
+  }
+  la.flush(wb);
   const int any_bad = __syncthreads_or((int)bad);
   for (int b = threadIdx.x; b < kBins; b += kThreads) {
     unsigned long long s = 0ull;
@@ -109,30 +180,41 @@ __device__ bool limb_any_below(const unsigned* L, int pos) {
   return off && (L[w] & ((1u << off) - 1u));
 }
 
+// Launched with one warp.  S = sum_b bin[b] 2^(b-1) (units of 2^-149) as a
+// 384-bit integer in 32-bit limbs: bin b = 32 li + bi + 1 adds bin << bi at
+// limb li.  Lane bi takes the bins 32 li + bi + 1 (li = 0..8) and adds the
+// three 32-bit parts of each shifted value to its limb sums (static indices:
+// registers); the lanes' limb sums are added over the warp in 64 bits
+// (< 2^39), and lane 0 carries them once and rounds.
 __global__ void absmean_finalize_kernel(AbsmeanWs* ws, int64_t n, float eps, float* gamma) {
+  constexpr int NL = 12;  // 384 bits: bins up to 287 (2^286 units) times 64-bit values, plus carries
+  const int lane = threadIdx.x & 31;
+  unsigned long long part[NL];
+#pragma unroll
+  for (int i = 0; i < NL; ++i) part[i] = 0ull;
+#pragma unroll
+  for (int li = 0; li < 9; ++li) {
+    const int b = 32 * li + lane + 1;
+    const unsigned long long v = b < kBins ? ws->bins[b] : 0ull;
+    const unsigned long long lo = v << lane;
+    const unsigned long long hi = lane ? (v >> (64 - lane)) : 0ull;
+    part[li] += lo & 0xFFFFFFFFull;
+    part[li + 1] += lo >> 32;
+    part[li + 2] += hi;
+  }
+#pragma unroll
+  for (int i = 0; i < NL; ++i)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part[i] += __shfl_xor_sync(0xFFFFFFFFu, part[i], o);
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
   if (ws->nonfinite) { *gamma = __int_as_float(0x7FC00000); return; }
-  constexpr int NL = 12;  // 384 bits >= 253 + 64 + carries
   unsigned L[NL];
+  unsigned long long carry = 0ull;
 #pragma unroll
-  for (int i = 0; i < NL; ++i) L[i] = 0u;
-  for (int e = 1; e < 255; ++e) {
-    const unsigned long long v = ws->bins[e];
-    if (!v) continue;
-    const int sh = e - 1;               // value = v * 2^(e-1) units of 2^-149
-    const int li = sh >> 5, bi = sh & 31;
-    // v << bi spans up to three limbs
-    unsigned long long lo = v << bi;
-    unsigned long long hi = bi ? (v >> (64 - bi)) : 0ull;
-    unsigned parts[3] = {(unsigned)lo, (unsigned)(lo >> 32), (unsigned)hi};
-    unsigned long long carry = 0ull;
-    for (int j = 0; li + j < NL; ++j) {
-      unsigned long long add = carry + (j < 3 ? parts[j] : 0u);
-      if (add == 0ull && j >= 3) break;
-      unsigned long long t = (unsigned long long)L[li + j] + add;
-      L[li + j] = (unsigned)t;
-      carry = t >> 32;
-    }
+  for (int i = 0; i < NL; ++i) {
+    const unsigned long long t = part[i] + carry;
+    L[i] = (unsigned)t;
+    carry = t >> 32;
   }
   int top = -1;
   for (int i = NL - 1; i >= 0 && top < 0; --i)
@@ -219,7 +301,7 @@ cudaError_t launch_absmean(const float* W, int64_t n, float eps, float* gamma, v
   AbsmeanWs* w = static_cast<AbsmeanWs*>(ws);
   cudaError_t e = cudaMemsetAsync(w, 0, sizeof(AbsmeanWs), s);
   if (e != cudaSuccess) return e;
-  absmean_bins_kernel<<<grid_for(n >> 2), kThreads, 0, s>>>(W, n, w);
+  absmean_bins_kernel<<<grid_for(n >> 4), kThreads, 0, s>>>(W, n, w);   // one block per 4 x 256 float4
   absmean_finalize_kernel<<<1, 32, 0, s>>>(w, n, eps, gamma);
   return cudaGetLastError();
 }

@@ -129,3 +129,22 @@ def test_tq1_all_243_codes_on_gpu():
     assert np.array_equal(qs.cpu().numpy(), qs_ref)
     assert len(set(qs_ref[:, :51].reshape(-1).tolist())) == 243
     assert np.array_equal(tri.unpack(qs, N, 256, "tq1").cpu().numpy(), trits)
+
+
+def test_absmean_exponent_window_paths():
+    """gamma bit-exact where the bins pass's per-warp exponent window has to
+    move up many times (magnitudes growing along W), where it starts high and
+    most later values fall below it (magnitudes shrinking), where warps start
+    on zeros, and where most values of a step sit far below its largest."""
+    rng = np.random.default_rng(17)
+    n = 64 * 4096
+    ramp = (rng.standard_normal(n) * np.exp2(np.linspace(-100, 100, n))).astype(np.float32)
+    half_zero = np.zeros(n, np.float32)
+    half_zero[n // 2:] = rng.standard_normal(n - n // 2).astype(np.float32) * 7
+    spikes = (rng.standard_normal(n) * 1e-12).astype(np.float32)
+    spikes[::37] = 1e30
+    for w in (ramp, ramp[::-1].copy(), half_zero, spikes):
+        W = w.reshape(64, 4096)
+        g_ref = O.absmean_gamma(W, 1e-6)
+        g = tri.absmean(torch.from_numpy(W).to(DEV), 1e-6)
+        assert _gamma_bits(g.item()) == _gamma_bits(g_ref)
