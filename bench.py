@@ -434,6 +434,79 @@ def measure_targets(args, rank, world, device):
     return out
 
 
+# ------------------------------------------------------------------ decode step (f3)
+DECODE_BLOCK = {"D": 8192, "H": 64, "Hkv": 8, "F": 28672}   # the 70B-like block's shapes
+
+
+def measure_decode_block(device, M=1, context=4096, steps=20, warmup=5, fmt="tq2"):
+    """One transformer-block decode step (RMSNorm, fused QKV, QK-Norm + RoPE
+    with cache append, grouped-query attention over `context` cached
+    positions, O, RMSNorm, fused gate/up SwiGLU, down, residuals) at the
+    70B-like shapes for M sequences, random ternary weights (P(0) = 0.31,
+    gamma 0.0159) and random caches; K steps captured in one CUDA graph and
+    timed with CUDA events.  Every step streams the block's packed weights
+    (220 MB TQ2) and the sequences' cached K and V (> L2), so no flush is
+    needed between steps."""
+    import bit_mixed_precision_tri_b200 as tri
+    from bit_mixed_precision_tri_b200 import decode as dec
+    from bit_mixed_precision_tri_b200 import inputs
+    Dm, H, Hkv, F = (DECODE_BLOCK[k] for k in ("D", "H", "Hkv", "F"))
+    hd = dec.HEAD_DIM
+    shapes = {"qkv": ((H + 2 * Hkv) * hd, Dm), "o": (Dm, H * hd), "gate": (F, Dm), "up": (F, Dm), "down": (Dm, F)}
+    w = {}
+    for i, (name, (n, k)) in enumerate(shapes.items()):
+        w[name] = (inputs.random_trits_on(device, n, k, 0.31, 200 + i),
+                   torch.tensor([0.0159], dtype=torch.float32, device=device))
+    for i, (name, n) in enumerate((("g_attn", Dm), ("g_mlp", Dm), ("gq", hd), ("gk", hd))):
+        w[name] = (1.0 + 0.25 * inputs.fp16_normal_on(device, (n,), 210 + i).float()).to(torch.float16)
+    Lmax = context + 1
+    blk = dec.DecodeBlock(w, Dm, H, Hkv, F, M, Lmax, device, fmt=fmt)
+    del w
+    blk.kcache.copy_(inputs.fp16_normal_on(device, tuple(blk.kcache.shape), 220))
+    blk.vcache.copy_(inputs.fp16_normal_on(device, tuple(blk.vcache.shape), 221))
+    x = inputs.fp16_normal_on(device, (M, Dm), 222)
+    pos = torch.full((M,), context, dtype=torch.int32, device=device)   # the new token follows `context` cached ones
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            blk.step(x, pos, context + 1)
+    torch.cuda.synchronize(device)
+    g_warm, g_steps = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_warm, stream=stream):
+        for _ in range(warmup):
+            blk.step(x, pos, context + 1)
+    with torch.cuda.graph(g_steps, stream=stream):
+        for _ in range(steps):
+            blk.step(x, pos, context + 1)
+    torch.cuda.synchronize(device)
+    g_warm.replay()
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        g_steps.replay()
+        t1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1) / steps
+    kv_bytes = M * Hkv * (context + 1) * hd * 2 * 2
+    act_bytes = 2 * M * (Dm * 12 + (H + 2 * Hkv) * hd + F * 3)           # fp16 activations in and out, roughly
+    step_bytes = blk.weight_bytes + kv_bytes + act_bytes
+    peaks, _ = load_peaks()
+    g = 1 if M <= 2 else 2                  # integer GEMM launches per call (3 <= M <= 16: prep + main)
+    # rmsnorm, qkv, qknorm_rope, attention (2), o, rmsnorm, gate/up SwiGLU (2), down, residual
+    launches = 1 + g + 1 + 2 + g + 1 + 2 + g + 1
+    res = {"M": M, "context": context, "fmt": fmt, "shapes": dict(DECODE_BLOCK, head_dim=hd),
+           "us_per_step": round(ms * 1e3, 2), "tokens_per_s": round(M / (ms * 1e-3), 1),
+           "bytes_per_step": step_bytes, "weight_bytes": blk.weight_bytes, "kv_bytes": kv_bytes,
+           "GB/s": round(step_bytes / (ms * 1e-3) / 1e9, 1),
+           "frac_of_hbm": round(step_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "steps": steps, "warmup": warmup, "gpu_launches_per_step": launches,
+           "data": "synthetic: random ternary weights (P(0) = 0.31), random fp16 caches and input"}
+    del blk
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ other rows
 def measure_rows(device, N=28672, K=8192, reps=5):
     """Time the offline rows of the path (absmean, ternarize, pack, unpack) on
@@ -639,6 +712,10 @@ def main():
                     help="skip the extra target workloads of the default line")
     ap.add_argument("--sweep", action="store_true",
                     help="print one line per batch-sweep, block and format-stress workload")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the one-block decode step (70B-like shapes, M = 1 and 16, "
+                         "4096 cached positions) and print it")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-step lines of the default run")
     ap.add_argument("--rows-only", action="store_true",
                     help="time only the offline rows (absmean, ternarize, pack, unpack) on the "
                          "28672x8192 weight, --steps timed calls each, and print them")
@@ -665,6 +742,12 @@ def main():
         if args.sweep:
             run_sweep(args, rank, world, device)
             return
+        if args.decode_only:
+            if rank == 0:
+                out = {f"decode_block70b_m{M}": measure_decode_block(device, M=M, steps=max(1, args.steps),
+                                                                     warmup=args.warmup) for M in (1, 16)}
+                print(json.dumps(out), flush=True)
+            return
         if args.rows_only:
             if rank == 0:
                 print(json.dumps({"rows": measure_rows(device, reps=max(1, args.steps))}), flush=True)
@@ -680,6 +763,10 @@ def main():
             res["targets"] = measure_targets(args, rank, world, device)
         if not args.no_rows:
             res["rows"] = measure_rows(device)
+        if not args.no_decode and args.workload == "down_8192x28672_m1" and args.M is None and args.fmt is None:
+            res["decode_block70b"] = {f"m{M}": measure_decode_block(device, M=M, steps=min(args.steps, 20),
+                                                                    warmup=max(3, min(args.warmup, 5)))
+                                      for M in (1, 16)}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             w = workload_from_args(args.workload, args.M, args.fmt)
             r = oracle_sample(w, budget_s=8.0)

@@ -52,6 +52,11 @@ SIGNATURES = {
     "tri_gemm_tq2_noalloc_fits": (_i, [_i64, _i64, _i64]),
     "tri_wait_status": (_i, [_p, _i, _p]),
     "tri_selftest_wait_timeout": (_i, [_i, _p, _p]),
+    "tri_rmsnorm": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _f, _p]),
+    "tri_rope_table": (_i, [_p, _i64, _i64, ctypes.c_double, _p]),
+    "tri_qknorm_rope": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _f, _p]),
+    "tri_attention_decode_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64]),
+    "tri_attention_decode": (_i, [_p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _p, _sz, _p]),
 }
 
 

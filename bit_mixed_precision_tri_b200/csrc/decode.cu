@@ -1,0 +1,366 @@
+// The non-linear steps of one transformer-block decode step around the
+// ternary linear layers ("Scaling Laws and Efficient Inference for Ternary
+// Language Models", section "The model": LLaMA-style blocks with SwiGLU,
+// rotary embeddings with theta = 5e5, RMSNorm and QK-Norm, no biases;
+// "Spectra: ...", section "Architecture of TriLM and FloatLM": activations
+// stay in 16-bit floats).  All activations are fp16 in HBM; arithmetic is
+// fp32; every kernel rounds once, where it stores.
+//
+//  * rmsnorm_kernel: y = x / sqrt(mean(x^2) + eps) * g per row, optionally
+//    after the residual sum h = x + r (fp16 add: the exact sum rounded once),
+//    which it stores too.  One CTA per row.
+//  * rope_table_kernel: (cos, sin) of p * theta^(-2i/dh) for every position p
+//    and pair i, angles in float64, stored as float32 pairs.
+//  * qknorm_rope_kernel: one warp per (token, head) of the fused QKV product:
+//    query and key heads are RMS-normalised over their 128 features (gains
+//    gq / gk) and rotated ("rotate half": pairs (i, i + 64)); the key and
+//    the value go into the caches at the token's position.  Lane l holds
+//    features 2l, 2l + 1, 64 + 2l, 65 + 2l: both members of its two pairs.
+//  * attn_decode_kernel: grouped-query attention of each sequence's new
+//    token over its cached positions 0..pos, split over positions.  A CTA
+//    owns (split, key/value head, sequence) and one warp per query head of
+//    the group; 64-position tiles of K and V are double-buffered in shared
+//    memory with cp.async (rows padded to 272 bytes: conflict-free 16-byte
+//    reads), scores and the running softmax are fp32, each lane owns four
+//    output features.  attn_combine_kernel merges the splits' (max, sum,
+//    output) triples.
+#include "tri_internal.cuh"
+
+namespace tri {
+namespace {
+
+constexpr int kDh = 128;            // head dimension served
+constexpr int kTP = 64;             // positions per attention tile
+constexpr int kRowB = 272;          // shared-memory row stride of K / V tiles, bytes
+constexpr int kAttnWarps = 8;       // query heads per key/value head served: up to 8
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// ---------------------------------------------------------------- RMSNorm
+__global__ void __launch_bounds__(256)
+rmsnorm_kernel(const __half* __restrict__ x, const __half* __restrict__ r, const __half* __restrict__ g,
+               __half* __restrict__ h_out, __half* __restrict__ y, int D, float eps) {
+  __shared__ float red[8];
+  const size_t row = (size_t)blockIdx.x * D;
+  const uint4* x8 = reinterpret_cast<const uint4*>(x + row);
+  const uint4* r8 = r ? reinterpret_cast<const uint4*>(r + row) : nullptr;
+  uint4* h8 = h_out ? reinterpret_cast<uint4*>(h_out + row) : nullptr;
+  const int n8 = D / 8;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+    uint4 v = x8[i];
+    if (r8) {
+      const uint4 w = r8[i];
+      __half2* a = reinterpret_cast<__half2*>(&v);
+      const __half2* b = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) a[k] = __hadd2(a[k], b[k]);   // exact sum, rounded once
+      h8[i] = v;
+    }
+    const __half2* a = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(a[k]);
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    }
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    t = warp_sum(t);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const float rstd = 1.f / sqrtf(red[0] / (float)D + eps);
+  const uint4* g8 = reinterpret_cast<const uint4*>(g);
+  uint4* y8 = reinterpret_cast<uint4*>(y + row);
+  for (int i = threadIdx.x; i < n8; i += blockDim.x) {
+    const uint4 v = h8 ? h8[i] : x8[i];      // h: written above by this thread
+    const uint4 gv = g8[i];
+    const __half2* a = reinterpret_cast<const __half2*>(&v);
+    const __half2* b = reinterpret_cast<const __half2*>(&gv);
+    uint4 o;
+    __half2* c = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __half22float2(a[k]), w = __half22float2(b[k]);
+      c[k] = __floats2half2_rn(f.x * rstd * w.x, f.y * rstd * w.y);
+    }
+    y8[i] = o;
+  }
+}
+
+// ---------------------------------------------------------------- RoPE table
+__global__ void rope_table_kernel(float2* __restrict__ cs, int Lmax, int half_dh, double theta) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)Lmax * half_dh) return;
+  const int p = (int)(idx / half_dh), i = (int)(idx % half_dh);
+  const double inv = pow(theta, -2.0 * (double)i / (double)(2 * half_dh));
+  double s, c;
+  sincos((double)p * inv, &s, &c);
+  cs[idx] = make_float2((float)c, (float)s);
+}
+
+// ---------------------------------------------------------------- QK-Norm + RoPE + cache append
+__global__ void __launch_bounds__(256)
+qknorm_rope_kernel(const __half* __restrict__ qkv, const int* __restrict__ pos, const __half* __restrict__ gq,
+                   const __half* __restrict__ gk, const float2* __restrict__ cs, __half* __restrict__ q_out,
+                   __half* __restrict__ kc, __half* __restrict__ vc, int M, int H, int Hkv, int Lmax, float eps) {
+  const int lane = threadIdx.x & 31;
+  const int nh = H + 2 * Hkv;
+  const int64_t wid = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (wid >= (int64_t)M * nh) return;
+  const int m = (int)(wid / nh), j = (int)(wid % nh);
+  const __half* src = qkv + ((size_t)m * nh + j) * kDh;
+  const __half2 a = *reinterpret_cast<const __half2*>(src + 2 * lane);
+  const __half2 b = *reinterpret_cast<const __half2*>(src + 64 + 2 * lane);
+  const int p = pos[m];
+  const bool in_range = p >= 0 && p < Lmax;            // else: nothing is cached, q unspecified
+  if (j >= H + Hkv) {                                  // value head: into the cache as is
+    if (in_range) {
+      __half* dst = vc + (((size_t)m * Hkv + (j - H - Hkv)) * Lmax + p) * kDh;
+      *reinterpret_cast<__half2*>(dst + 2 * lane) = a;
+      *reinterpret_cast<__half2*>(dst + 64 + 2 * lane) = b;
+    }
+    return;
+  }
+  const float2 fa = __half22float2(a), fb = __half22float2(b);
+  const float ss = warp_sum(fa.x * fa.x + fa.y * fa.y + fb.x * fb.x + fb.y * fb.y);
+  const float rstd = 1.f / sqrtf(ss / (float)kDh + eps);
+  const __half* g = j < H ? gq : gk;
+  const float2 ga = __half22float2(*reinterpret_cast<const __half2*>(g + 2 * lane));
+  const float2 gb = __half22float2(*reinterpret_cast<const __half2*>(g + 64 + 2 * lane));
+  const float x0 = fa.x * rstd * ga.x, x1 = fa.y * rstd * ga.y;    // features 2l, 2l + 1
+  const float y0 = fb.x * rstd * gb.x, y1 = fb.y * rstd * gb.y;    // features 64 + 2l, 65 + 2l
+  const int pc = in_range ? p : 0;
+  const float2 c0 = cs[(size_t)pc * 64 + 2 * lane], c1 = cs[(size_t)pc * 64 + 2 * lane + 1];
+  const __half2 oa = __floats2half2_rn(x0 * c0.x - y0 * c0.y, x1 * c1.x - y1 * c1.y);
+  const __half2 ob = __floats2half2_rn(y0 * c0.x + x0 * c0.y, y1 * c1.x + x1 * c1.y);
+  __half* dst;
+  if (j < H) {
+    dst = q_out + ((size_t)m * H + j) * kDh;
+  } else {
+    if (!in_range) return;
+    dst = kc + (((size_t)m * Hkv + (j - H)) * Lmax + p) * kDh;
+  }
+  *reinterpret_cast<__half2*>(dst + 2 * lane) = oa;
+  *reinterpret_cast<__half2*>(dst + 64 + 2 * lane) = ob;
+}
+
+// ---------------------------------------------------------------- attention
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src, uint32_t n) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ uint32_t s_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+constexpr int kTileBytes = kTP * kRowB;                                    // one K or V tile
+constexpr int kAttnSmem = 2 * 2 * kTileBytes + kAttnWarps * kDh * 2 + kAttnWarps * kTP * 4;
+static_assert(kTP * 16 % 256 == 0, "whole copies per thread");
+
+// grid (splits, Hkv, M); warp w serves query head kvh * G + w (w < G)
+__global__ void __launch_bounds__(256)
+attn_decode_kernel(const __half* __restrict__ q, const __half* __restrict__ kc, const __half* __restrict__ vc,
+                   const int* __restrict__ pos, float* __restrict__ part_o, float2* __restrict__ part_ml,
+                   int H, int Hkv, int Lmax, int max_len, int tiles_per_split) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint8_t* qsm = sm + 4 * kTileBytes;                                    // [G][128] fp16
+  float* psm = reinterpret_cast<float*>(qsm + kAttnWarps * kDh * 2);     // [G][64]
+  const int s = blockIdx.x, kvh = blockIdx.y, m = blockIdx.z, splits = gridDim.x;
+  const int G = H / Hkv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int L = pos[m] + 1;                                  // clamped to [1, max_len] (max_len <= Lmax)
+  L = L < 1 ? 1 : (L > max_len ? max_len : L);
+  const int t0 = s * tiles_per_split * kTP;
+  const int t1 = min(L, t0 + tiles_per_split * kTP);
+  const int ntiles = t1 > t0 ? (t1 - t0 + kTP - 1) / kTP : 0;
+  // this group's query vectors
+  for (int i = threadIdx.x; i < G * 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(qsm)[i] =
+        reinterpret_cast<const uint4*>(q + ((size_t)m * H + (size_t)kvh * G) * kDh)[i];
+  const __half* kb = kc + ((size_t)m * Hkv + kvh) * Lmax * kDh;
+  const __half* vb = vc + ((size_t)m * Hkv + kvh) * Lmax * kDh;
+  // tile `it` into buffer it & 1: 64 rows x 16 chunks of K and of V, i.e.
+  // 1024 chunks each, 4 + 4 copies per thread (rows 0..63, chunks 0..15)
+  auto issue = [&](int it) {
+    const int base = t0 + it * kTP;
+    uint8_t* kt = sm + (it & 1) * 2 * kTileBytes;
+#pragma unroll
+    for (int c = 0; c < kTP * 16 / 256; ++c) {
+      const int idx = c * 256 + threadIdx.x, row = idx >> 4, col = idx & 15;
+      const bool ok = base + row < t1;
+      const size_t off = (size_t)(ok ? base + row : 0) * kDh + col * 8;
+      cp16(s_addr(kt + row * kRowB + col * 16), kb + off, ok ? 16u : 0u);
+      cp16(s_addr(kt + kTileBytes + row * kRowB + col * 16), vb + off, ok ? 16u : 0u);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  if (ntiles > 0) issue(0);
+  __syncthreads();                                     // q staged
+  const float scale = rsqrtf((float)kDh);
+  float mrun = -INFINITY, lrun = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int it = 0; it < ntiles; ++it) {
+    if (it + 1 < ntiles) {
+      issue(it + 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    __syncthreads();
+    const uint8_t* kt = sm + (it & 1) * 2 * kTileBytes;
+    const uint8_t* vt = kt + kTileBytes;
+    const int base = t0 + it * kTP;
+    if (warp < G) {
+      const uint4* qv = reinterpret_cast<const uint4*>(qsm + warp * kDh * 2);
+      float sc[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int pl = lane + 32 * r;
+        const uint4* kr = reinterpret_cast<const uint4*>(kt + pl * kRowB);
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint4 kk = kr[c], qq = qv[c];
+          const __half2* k2 = reinterpret_cast<const __half2*>(&kk);
+          const __half2* q2 = reinterpret_cast<const __half2*>(&qq);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fk = __half22float2(k2[e]), fq = __half22float2(q2[e]);
+            dot = fmaf(fk.x, fq.x, fmaf(fk.y, fq.y, dot));
+          }
+        }
+        sc[r] = base + pl < t1 ? dot * scale : -INFINITY;
+      }
+      const float mnew = fmaxf(mrun, warp_max(fmaxf(sc[0], sc[1])));
+      const float alpha = expf(mrun - mnew);           // 0 while mrun is -inf
+      const float p0 = expf(sc[0] - mnew), p1 = expf(sc[1] - mnew);
+      lrun = lrun * alpha + warp_sum(p0 + p1);
+      mrun = mnew;
+      float* pw = psm + warp * kTP;
+      pw[lane] = p0;
+      pw[lane + 32] = p1;
+      __syncwarp();
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[e] *= alpha;
+#pragma unroll 8
+      for (int pl = 0; pl < kTP; ++pl) {
+        const float pv = pw[pl];
+        const uint2 vv = *reinterpret_cast<const uint2*>(vt + pl * kRowB + lane * 8);
+        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
+        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
+        o[0] = fmaf(pv, v01.x, o[0]);
+        o[1] = fmaf(pv, v01.y, o[1]);
+        o[2] = fmaf(pv, v23.x, o[2]);
+        o[3] = fmaf(pv, v23.y, o[3]);
+      }
+      __syncwarp();
+    }
+    __syncthreads();                                   // the buffer may be refilled
+  }
+  if (warp < G) {
+    const size_t slot = ((size_t)m * H + (size_t)kvh * G + warp) * splits + s;
+    *reinterpret_cast<float4*>(part_o + slot * kDh + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+    if (lane == 0) part_ml[slot] = make_float2(mrun, lrun);
+  }
+}
+
+// one CTA of 128 threads per (sequence, query head): sum over the splits
+__global__ void __launch_bounds__(128)
+attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml, __half* __restrict__ out,
+                    int splits) {
+  const size_t mh = blockIdx.x;
+  const int d = threadIdx.x;
+  float mx = -INFINITY;
+  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_ml[mh * splits + s].x);
+  float l = 0.f, acc = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float2 ml = part_ml[mh * splits + s];
+    const float w = ml.y > 0.f ? expf(ml.x - mx) : 0.f;
+    l = fmaf(w, ml.y, l);
+    acc = fmaf(w, part_o[(mh * splits + s) * kDh + d], acc);
+  }
+  out[mh * kDh + d] = __float2half_rn(acc / l);
+}
+
+struct AttnPlan {
+  int splits, tiles_per_split;
+  size_t off_ml, total;
+};
+
+AttnPlan attn_plan(int64_t M, int64_t H, int64_t Hkv, int64_t max_len, int sms) {
+  AttnPlan pl;
+  const int64_t tiles = (max_len + kTP - 1) / kTP;
+  int64_t sp = (2 * (int64_t)sms + M * Hkv - 1) / (M * Hkv);   // about two CTAs per SM
+  if (sp > tiles) sp = tiles;
+  if (sp < 1) sp = 1;
+  pl.tiles_per_split = (int)((tiles + sp - 1) / sp);
+  pl.splits = (int)((tiles + pl.tiles_per_split - 1) / pl.tiles_per_split);
+  const size_t n = (size_t)M * H * pl.splits;
+  pl.off_ml = (n * kDh * 4 + 255) & ~size_t(255);
+  pl.total = pl.off_ml + ((n * 8 + 255) & ~size_t(255));
+  return pl;
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm(const __half* x, const __half* r, const __half* g, __half* h_out, __half* y,
+                           int64_t M, int64_t D, float eps, cudaStream_t s) {
+  rmsnorm_kernel<<<(unsigned)M, 256, 0, s>>>(x, r, g, h_out, y, (int)D, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(float2* cs, int64_t Lmax, int64_t dh, double theta, cudaStream_t s) {
+  const int64_t n = Lmax * (dh / 2);
+  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(cs, (int)Lmax, (int)(dh / 2), theta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qknorm_rope(const __half* qkv, const int* pos, const __half* gq, const __half* gk,
+                               const float2* cs, __half* q_out, __half* kc, __half* vc, int64_t M, int64_t H,
+                               int64_t Hkv, int64_t Lmax, float eps, cudaStream_t s) {
+  const int64_t warps = M * (H + 2 * Hkv);
+  qknorm_rope_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(qkv, pos, gq, gk, cs, q_out, kc, vc, (int)M,
+                                                                  (int)H, (int)Hkv, (int)Lmax, eps);
+  return cudaGetLastError();
+}
+
+size_t attention_decode_ws_bytes(int64_t M, int64_t H, int64_t Hkv, int64_t max_len, int sms) {
+  return attn_plan(M, H, Hkv, max_len, sms).total;
+}
+
+cudaError_t launch_attention_decode(const __half* q, const __half* kc, const __half* vc, const int* pos,
+                                    __half* out, int64_t M, int64_t H, int64_t Hkv, int64_t Lmax,
+                                    int64_t max_len, void* ws, int sms, cudaStream_t s) {
+  const AttnPlan pl = attn_plan(M, H, Hkv, max_len, sms);
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               kAttnSmem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_done[dev] = true;
+  }
+  float* part_o = static_cast<float*>(ws);
+  float2* part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + pl.off_ml);
+  attn_decode_kernel<<<dim3((unsigned)pl.splits, (unsigned)Hkv, (unsigned)M), 256, kAttnSmem, s>>>(
+      q, kc, vc, pos, part_o, part_ml, (int)H, (int)Hkv, (int)Lmax, (int)max_len, pl.tiles_per_split);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_combine_kernel<<<(unsigned)(M * H), kDh, 0, s>>>(part_o, part_ml, out, pl.splits);
+  return cudaGetLastError();
+}
+
+}  // namespace tri

@@ -89,6 +89,14 @@ size_t path_ws_bytes(int fmt, int path, int64_t M, int64_t N, int64_t K, int sms
   return transcode_bytes(fmt, path, M, N, K) + inner;
 }
 
+// shapes the decode-step attention serves
+tri_status attn_shape(int64_t M, int64_t H, int64_t Hkv, int64_t Lmax, int64_t max_len) {
+  if (M < 1 || M > 65535 || H < 1 || Hkv < 1 || Hkv > 65535 || H % Hkv != 0 || H / Hkv > 8) return TRI_ERR_SHAPE;
+  if (Lmax < 1 || Lmax > (int64_t(1) << 24) || max_len < 1 || max_len > Lmax) return TRI_ERR_SHAPE;
+  if (M * Hkv * Lmax > (int64_t(1) << 40) / 128 || M * H > (int64_t(1) << 31) - 1) return TRI_ERR_SHAPE;
+  return TRI_OK;
+}
+
 int auto_path(int fmt, int64_t M, int64_t N, int64_t K) {
   if (M <= 16 && path_supported(fmt, TRI_PATH_I8, M, N, K)) return TRI_PATH_I8;
   if (M <= 16 && path_supported(fmt, TRI_PATH_MMA, M, N, K)) return TRI_PATH_MMA;
@@ -386,6 +394,83 @@ tri_status tri_gemm_tq1(const uint16_t* X, const uint8_t* qs, const uint16_t* d,
                         int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                         void* stream) {
   return tri_gemm(TRI_TQ1, TRI_PATH_AUTO, X, qs, d, Y, M, N, K, workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------- decode step
+tri_status tri_rmsnorm(const uint16_t* x, const uint16_t* r, const uint16_t* g, uint16_t* h_out, uint16_t* y,
+                       int64_t M, int64_t D, float eps, void* stream) {
+  if (!x || !g || !y || (r && !h_out)) return TRI_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(eps < 1e30f)) return TRI_ERR_INVALID_ARG;
+  if (r && (h_out == x || h_out == r)) return TRI_ERR_INVALID_ARG;
+  if (M < 1 || M > kMaxDim || D < 8 || D > (int64_t(1) << 20) || D % 8 != 0) return TRI_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(g, 16) || !aligned(y, 16) || (r && !aligned(r, 16)) ||
+      (h_out && !aligned(h_out, 16)))
+    return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  tri_status st = device_info(&di);
+  if (st != TRI_OK) return st;
+  return from_cuda(tri::launch_rmsnorm(reinterpret_cast<const __half*>(x), reinterpret_cast<const __half*>(r),
+                                       reinterpret_cast<const __half*>(g), r ? reinterpret_cast<__half*>(h_out) : nullptr,
+                                       reinterpret_cast<__half*>(y), M, D, eps, static_cast<cudaStream_t>(stream)));
+}
+
+tri_status tri_rope_table(float* cs, int64_t Lmax, int64_t dh, double theta, void* stream) {
+  if (!cs || !(theta > 1.0) || !(theta < 1e300)) return TRI_ERR_INVALID_ARG;
+  if (dh != 128 || Lmax < 1 || Lmax > (int64_t(1) << 24)) return TRI_ERR_SHAPE;
+  if (!aligned(cs, 8)) return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  tri_status st = device_info(&di);
+  if (st != TRI_OK) return st;
+  return from_cuda(tri::launch_rope_table(reinterpret_cast<float2*>(cs), Lmax, dh, theta,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+tri_status tri_qknorm_rope(const uint16_t* qkv, const int32_t* pos, const uint16_t* gq, const uint16_t* gk,
+                           const float* cs, uint16_t* q_out, uint16_t* kcache, uint16_t* vcache, int64_t M,
+                           int64_t H, int64_t Hkv, int64_t Lmax, float eps, void* stream) {
+  if (!qkv || !pos || !gq || !gk || !cs || !q_out || !kcache || !vcache) return TRI_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(eps < 1e30f)) return TRI_ERR_INVALID_ARG;
+  if (M < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || Lmax < 1 || Lmax > (int64_t(1) << 24)) return TRI_ERR_SHAPE;
+  if (M * (H + 2 * Hkv) > kMaxDim || M * Hkv * Lmax > (int64_t(1) << 40) / 128) return TRI_ERR_SHAPE;
+  if (!aligned(qkv, 16) || !aligned(gq, 16) || !aligned(gk, 16) || !aligned(q_out, 16) ||
+      !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(pos, 4) || !aligned(cs, 8))
+    return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  tri_status st = device_info(&di);
+  if (st != TRI_OK) return st;
+  return from_cuda(tri::launch_qknorm_rope(
+      reinterpret_cast<const __half*>(qkv), pos, reinterpret_cast<const __half*>(gq),
+      reinterpret_cast<const __half*>(gk), reinterpret_cast<const float2*>(cs), reinterpret_cast<__half*>(q_out),
+      reinterpret_cast<__half*>(kcache), reinterpret_cast<__half*>(vcache), M, H, Hkv, Lmax, eps,
+      static_cast<cudaStream_t>(stream)));
+}
+
+size_t tri_attention_decode_workspace_bytes(int64_t M, int64_t H, int64_t Hkv, int64_t max_len) {
+  if (attn_shape(M, H, Hkv, max_len, max_len) != TRI_OK) return 0;
+  DevInfo di;
+  int sms = 148;
+  if (device_info(&di) == TRI_OK) sms = di.sms;
+  return tri::attention_decode_ws_bytes(M, H, Hkv, max_len, sms);
+}
+
+tri_status tri_attention_decode(const uint16_t* q, const uint16_t* kcache, const uint16_t* vcache,
+                                const int32_t* pos, uint16_t* out, int64_t M, int64_t H, int64_t Hkv,
+                                int64_t Lmax, int64_t max_len, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  if (!q || !kcache || !vcache || !pos || !out) return TRI_ERR_INVALID_ARG;
+  tri_status st = attn_shape(M, H, Hkv, Lmax, max_len);
+  if (st != TRI_OK) return st;
+  if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(out, 16) || !aligned(pos, 4))
+    return TRI_ERR_ALIGNMENT;
+  DevInfo di;
+  if ((st = device_info(&di)) != TRI_OK) return st;
+  const size_t need = tri::attention_decode_ws_bytes(M, H, Hkv, max_len, di.sms);
+  if (!workspace || workspace_bytes < need) return TRI_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return TRI_ERR_ALIGNMENT;
+  return from_cuda(tri::launch_attention_decode(
+      reinterpret_cast<const __half*>(q), reinterpret_cast<const __half*>(kcache),
+      reinterpret_cast<const __half*>(vcache), pos, reinterpret_cast<__half*>(out), M, H, Hkv, Lmax, max_len,
+      workspace, di.sms, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -64,6 +64,18 @@ size_t gemv_i8_ws_bytes(int64_t M, int64_t N, int64_t K, int num_sms, bool tq1 =
 cudaError_t launch_gemv_i8(const __half* X, const uint8_t* qs, const __half* d, __half* Y, int M,
                            int N, int K, void* ws, int num_sms, cudaStream_t s, bool tq1 = false);
 
+// one-block decode step around the ternary layers (decode.cu); head dim 128
+cudaError_t launch_rmsnorm(const __half* x, const __half* r, const __half* g, __half* h_out, __half* y,
+                           int64_t M, int64_t D, float eps, cudaStream_t s);
+cudaError_t launch_rope_table(float2* cs, int64_t Lmax, int64_t dh, double theta, cudaStream_t s);
+cudaError_t launch_qknorm_rope(const __half* qkv, const int* pos, const __half* gq, const __half* gk,
+                               const float2* cs, __half* q_out, __half* kc, __half* vc, int64_t M, int64_t H,
+                               int64_t Hkv, int64_t Lmax, float eps, cudaStream_t s);
+size_t attention_decode_ws_bytes(int64_t M, int64_t H, int64_t Hkv, int64_t max_len, int sms);
+cudaError_t launch_attention_decode(const __half* q, const __half* kc, const __half* vc, const int* pos,
+                                    __half* out, int64_t M, int64_t H, int64_t Hkv, int64_t Lmax,
+                                    int64_t max_len, void* ws, int sms, cudaStream_t s);
+
 // decode-regime path with library-owned static scratch (no allocation)
 size_t gemv_noalloc_scratch_limit();
 size_t gemv_noalloc_scratch_need(int64_t M, int64_t N, int64_t K, int num_sms);

@@ -51,3 +51,20 @@ def random_bytes(n: int, seed: int) -> torch.Tensor:
 
 def as_numpy(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
+
+
+def random_trits_on(device, N: int, K: int, p_zero: float, seed: int) -> torch.Tensor:
+    """As ``random_trits``, drawn by torch's generator on `device` (for large
+    timing-only weights; the parity tests use the CPU draws)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    u = torch.rand(N, K, generator=g, device=device)
+    s = torch.randint(0, 2, (N, K), generator=g, dtype=torch.int8, device=device) * 2 - 1
+    return torch.where(u < p_zero, torch.zeros_like(s), s).to(torch.int8)
+
+
+def fp16_normal_on(device, shape, seed: int, std: float = 1.0) -> torch.Tensor:
+    """fp16 tensor ~ N(0, std) drawn on `device` (timing-only caches)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return (torch.randn(*shape, generator=g, device=device) * std).to(torch.float16)

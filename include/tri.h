@@ -290,6 +290,60 @@ TRI_API tri_status tri_selftest_wait_timeout(int which, void* scratch, void* str
  * (one of tri_gemm_path), or -1 if the shape is invalid. */
 TRI_API int tri_gemm_auto_path(int format, int64_t M, int64_t N, int64_t K);
 
+/* ----------------------------------------------------------------------
+ * One transformer-block decode step around the ternary layers
+ * ("Scaling Laws and Efficient Inference for Ternary Language Models",
+ * section "The model": LLaMA-style blocks with SwiGLU MLPs, rotary
+ * embeddings with theta = 5e5, RMSNorm and QK-Norm, no biases; "Spectra:
+ * ...", section "Architecture of TriLM and FloatLM": activations in 16-bit
+ * floats).  The linear layers of the block are tri_gemm / tri_gemm_swiglu
+ * calls; these entry points are the steps between them.  All tensors are
+ * caller-owned device memory, fp16 unless stated, row-major, 16-byte
+ * aligned (pos: 4, cs: 8); arithmetic is fp32 and each result is rounded
+ * to fp16 once, where it is stored.  Head dimension 128 throughout.
+ *
+ * tri_rmsnorm: y[m] = h[m] / sqrt(mean(h[m]^2) + eps) * g, where h = x, or,
+ *   when r is not NULL, h = x + r (each element the exact sum rounded once),
+ *   which is also written to h_out (required then; it may not alias x or r).
+ *   x, r, h_out, y: [M][D]; g: [D]; 8 <= D <= 2^20, D % 8 == 0, M >= 1,
+ *   0 <= eps < 1e30.  y may alias x when r is NULL.
+ * tri_rope_table: cs[p][i] = (cos, sin)(p * theta^(-2 i / dh)) as float
+ *   pairs for p < Lmax, i < dh / 2, the angles computed in float64
+ *   (rotate-half RoPE: pair i is (feature i, feature i + dh / 2)); dh = 128,
+ *   1 <= Lmax <= 2^24, theta > 1.
+ * tri_qknorm_rope: qkv [M][(H + 2 Hkv) * 128] is the fused QKV product
+ *   (query heads, then key heads, then value heads).  Each query and key
+ *   head is RMS-normalised over its 128 features with gain gq or gk ([128],
+ *   shared by the heads) and rotated at position pos[m] with the table cs
+ *   ([>= Lmax][64] float pairs); queries go to q_out [M][H][128], the key
+ *   and the value (as given) to kcache / vcache [M][Hkv][Lmax][128] at
+ *   position pos[m] (device int32 [M]).  A position outside [0, Lmax)
+ *   writes nothing to the caches and leaves that q unspecified.  H % Hkv == 0.
+ * tri_attention_decode: out[m][h] = softmax(K q[m][h] / sqrt(128)) V over
+ *   positions 0..pos[m] of sequence m's caches, key/value head h / (H / Hkv)
+ *   (grouped queries, H / Hkv <= 8); out: [M][H * 128].  max_len (host) is
+ *   an upper bound of pos[m] + 1 over the batch, 1 <= max_len <= Lmax: it
+ *   sizes the split over positions and the workspace
+ *   (tri_attention_decode_workspace_bytes, 256-byte aligned, contents on
+ *   entry irrelevant); a pos[m] + 1 above max_len is clamped to it.  Calls
+ *   that share a workspace must be ordered.
+ * Errors: TRI_ERR_INVALID_ARG (null pointer, eps or theta out of range,
+ *   missing h_out), TRI_ERR_SHAPE, TRI_ERR_ALIGNMENT, TRI_ERR_WORKSPACE,
+ *   TRI_ERR_CUDA; nothing traps.
+ * ---------------------------------------------------------------------- */
+TRI_API tri_status tri_rmsnorm(const uint16_t* x, const uint16_t* r, const uint16_t* g, uint16_t* h_out,
+                               uint16_t* y, int64_t M, int64_t D, float eps, void* stream);
+TRI_API tri_status tri_rope_table(float* cs, int64_t Lmax, int64_t dh, double theta, void* stream);
+TRI_API tri_status tri_qknorm_rope(const uint16_t* qkv, const int32_t* pos, const uint16_t* gq,
+                                   const uint16_t* gk, const float* cs, uint16_t* q_out, uint16_t* kcache,
+                                   uint16_t* vcache, int64_t M, int64_t H, int64_t Hkv, int64_t Lmax,
+                                   float eps, void* stream);
+TRI_API size_t tri_attention_decode_workspace_bytes(int64_t M, int64_t H, int64_t Hkv, int64_t max_len);
+TRI_API tri_status tri_attention_decode(const uint16_t* q, const uint16_t* kcache, const uint16_t* vcache,
+                                        const int32_t* pos, uint16_t* out, int64_t M, int64_t H,
+                                        int64_t Hkv, int64_t Lmax, int64_t max_len, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
