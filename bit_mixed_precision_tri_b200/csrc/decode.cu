@@ -167,39 +167,71 @@ __device__ __forceinline__ uint32_t s_addr(const void* p) {
 }
 
 constexpr int kTileBytes = kTP * kRowB;                                    // one K or V tile
-constexpr int kAttnSmem = 2 * 2 * kTileBytes + kAttnWarps * kDh * 2 + kAttnWarps * kTP * 4;
-static_assert(kTP * 16 % 256 == 0, "whole copies per thread");
+constexpr int kAttnThreads = 128;                                          // 4 warps x 16 positions
+constexpr int kAttnParts = kAttnThreads / 32;                              // partial results per split
+constexpr int kAttnSmem = 2 * 2 * kTileBytes + kAttnWarps * kDh * 2;
+static_assert(kTP == 16 * kAttnParts, "one 16-position slice per warp");
+static_assert(kTP * 16 % kAttnThreads == 0, "whole copies per thread");
 
-// grid (splits, Hkv, M); warp w serves query head kvh * G + w (w < G)
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  // rows 8..15 of A are zero (at most 8 query heads per group)
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr) : "memory");
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// grid (splits, Hkv, M), 4 warps.  The group's G <= 8 query heads are the
+// rows of the MMAs' A operand (rows 8..15 zero).  Warp w takes positions
+// 16w .. 16w + 15 of every 64-position tile: S = Q K^T over them (two n8
+// tiles, eight k16 steps, the B fragments read straight from the K tile:
+// lane (gid, tig) reads position gid, features 2 tig, 2 tig + 1 (+8), which
+// hit 32 distinct banks with 272-byte rows), the running softmax per head
+// row (the four lanes of a quad hold a row), then O += P V with P taken from
+// the S accumulators as the A operand and V's B fragments by ldmatrix.trans.
+// Each warp leaves its own (max, sum, output) partial.
+__global__ void __launch_bounds__(kAttnThreads)
 attn_decode_kernel(const __half* __restrict__ q, const __half* __restrict__ kc, const __half* __restrict__ vc,
                    const int* __restrict__ pos, float* __restrict__ part_o, float2* __restrict__ part_ml,
                    int H, int Hkv, int Lmax, int max_len, int tiles_per_split) {
   extern __shared__ __align__(16) uint8_t sm[];
   uint8_t* qsm = sm + 4 * kTileBytes;                                    // [G][128] fp16
-  float* psm = reinterpret_cast<float*>(qsm + kAttnWarps * kDh * 2);     // [G][64]
   const int s = blockIdx.x, kvh = blockIdx.y, m = blockIdx.z, splits = gridDim.x;
   const int G = H / Hkv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
   int L = pos[m] + 1;                                  // clamped to [1, max_len] (max_len <= Lmax)
   L = L < 1 ? 1 : (L > max_len ? max_len : L);
   const int t0 = s * tiles_per_split * kTP;
   const int t1 = min(L, t0 + tiles_per_split * kTP);
   const int ntiles = t1 > t0 ? (t1 - t0 + kTP - 1) / kTP : 0;
-  // this group's query vectors
-  for (int i = threadIdx.x; i < G * 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < G * 16; i += kAttnThreads)
     reinterpret_cast<uint4*>(qsm)[i] =
         reinterpret_cast<const uint4*>(q + ((size_t)m * H + (size_t)kvh * G) * kDh)[i];
   const __half* kb = kc + ((size_t)m * Hkv + kvh) * Lmax * kDh;
   const __half* vb = vc + ((size_t)m * Hkv + kvh) * Lmax * kDh;
   // tile `it` into buffer it & 1: 64 rows x 16 chunks of K and of V, i.e.
-  // 1024 chunks each, 4 + 4 copies per thread (rows 0..63, chunks 0..15)
+  // 1024 chunks each, 8 + 8 copies per thread (rows 0..63, chunks 0..15)
   auto issue = [&](int it) {
     const int base = t0 + it * kTP;
     uint8_t* kt = sm + (it & 1) * 2 * kTileBytes;
 #pragma unroll
-    for (int c = 0; c < kTP * 16 / 256; ++c) {
-      const int idx = c * 256 + threadIdx.x, row = idx >> 4, col = idx & 15;
+    for (int c = 0; c < kTP * 16 / kAttnThreads; ++c) {
+      const int idx = c * kAttnThreads + threadIdx.x, row = idx >> 4, col = idx & 15;
       const bool ok = base + row < t1;
       const size_t off = (size_t)(ok ? base + row : 0) * kDh + col * 8;
       cp16(s_addr(kt + row * kRowB + col * 16), kb + off, ok ? 16u : 0u);
@@ -209,8 +241,22 @@ attn_decode_kernel(const __half* __restrict__ q, const __half* __restrict__ kc, 
   };
   if (ntiles > 0) issue(0);
   __syncthreads();                                     // q staged
+  // A fragments of Q: row gid (a query head, zero past G), k step kk:
+  // features 16 kk + 2 tig, +1 (a0) and 16 kk + 8 + 2 tig, +1 (a2)
+  uint32_t qa[8][2];
+  {
+    const uint32_t qrow = s_addr(qsm) + (uint32_t)gid * kDh * 2 + 4 * tig;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      qa[kk][0] = gid < G ? lds_u32(qrow + 32 * kk) : 0u;
+      qa[kk][1] = gid < G ? lds_u32(qrow + 32 * kk + 16) : 0u;
+    }
+  }
   const float scale = rsqrtf((float)kDh);
-  float mrun = -INFINITY, lrun = 0.f, o[4] = {0.f, 0.f, 0.f, 0.f};
+  float mrun = -INFINITY, lrun = 0.f;
+  float o[16][4];
+#pragma unroll
+  for (int nf = 0; nf < 16; ++nf) o[nf][0] = o[nf][1] = o[nf][2] = o[nf][3] = 0.f;
   for (int it = 0; it < ntiles; ++it) {
     if (it + 1 < ntiles) {
       issue(it + 1);
@@ -219,60 +265,80 @@ attn_decode_kernel(const __half* __restrict__ q, const __half* __restrict__ kc, 
       asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
-    const uint8_t* kt = sm + (it & 1) * 2 * kTileBytes;
-    const uint8_t* vt = kt + kTileBytes;
-    const int base = t0 + it * kTP;
-    if (warp < G) {
-      const uint4* qv = reinterpret_cast<const uint4*>(qsm + warp * kDh * 2);
-      float sc[2];
+    const uint32_t kt = s_addr(sm + (it & 1) * 2 * kTileBytes) + 16 * warp * kRowB;   // this warp's 16 rows
+    const uint32_t vt = kt + kTileBytes;
+    const int p0 = t0 + it * kTP + 16 * warp;          // position of the warp's first row
+    // S = Q K^T: n tile nt = positions p0 + 8 nt .. + 7
+    float sacc[2][4];
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int pl = lane + 32 * r;
-        const uint4* kr = reinterpret_cast<const uint4*>(kt + pl * kRowB);
-        float dot = 0.f;
+    for (int nt = 0; nt < 2; ++nt) {
+      sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      const uint32_t krow = kt + (uint32_t)(8 * nt + gid) * kRowB + 4 * tig;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const uint4 kk = kr[c], qq = qv[c];
-          const __half2* k2 = reinterpret_cast<const __half2*>(&kk);
-          const __half2* q2 = reinterpret_cast<const __half2*>(&qq);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_f16(sacc[nt], qa[kk][0], qa[kk][1], lds_u32(krow + 32 * kk), lds_u32(krow + 32 * kk + 16));
+    }
+    // row gid's scores at positions p0 + 8 nt + 2 tig + e
+    float sc[2][2];
+    float mt = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 fk = __half22float2(k2[e]), fq = __half22float2(q2[e]);
-            dot = fmaf(fk.x, fq.x, fmaf(fk.y, fq.y, dot));
-          }
-        }
-        sc[r] = base + pl < t1 ? dot * scale : -INFINITY;
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        sc[nt][e] = p0 + 8 * nt + 2 * tig + e < t1 ? sacc[nt][e] * scale : -INFINITY;
+        mt = fmaxf(mt, sc[nt][e]);
       }
-      const float mnew = fmaxf(mrun, warp_max(fmaxf(sc[0], sc[1])));
-      const float alpha = expf(mrun - mnew);           // 0 while mrun is -inf
-      const float p0 = expf(sc[0] - mnew), p1 = expf(sc[1] - mnew);
-      lrun = lrun * alpha + warp_sum(p0 + p1);
-      mrun = mnew;
-      float* pw = psm + warp * kTP;
-      pw[lane] = p0;
-      pw[lane + 32] = p1;
-      __syncwarp();
+    mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, 1));
+    mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, 2));
+    const float mnew = fmaxf(mrun, mt);
+    // no valid position seen yet (a slice past the end): nothing changes
+    const float alpha = mnew == -INFINITY ? 1.f : expf(mrun - mnew);
+    float pr[2][2], ps = 0.f;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] *= alpha;
-#pragma unroll 8
-      for (int pl = 0; pl < kTP; ++pl) {
-        const float pv = pw[pl];
-        const uint2 vv = *reinterpret_cast<const uint2*>(vt + pl * kRowB + lane * 8);
-        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&vv.x));
-        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&vv.y));
-        o[0] = fmaf(pv, v01.x, o[0]);
-        o[1] = fmaf(pv, v01.y, o[1]);
-        o[2] = fmaf(pv, v23.x, o[2]);
-        o[3] = fmaf(pv, v23.y, o[3]);
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        pr[nt][e] = mnew == -INFINITY ? 0.f : expf(sc[nt][e] - mnew);
+        ps += pr[nt][e];
       }
-      __syncwarp();
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 1);
+    ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 2);
+    lrun = lrun * alpha + ps;
+    mrun = mnew;
+    // O = alpha O + P V: A = P (row gid, k = positions 2 tig, +1 and 8 + 2 tig, +1)
+    // as two fp16 parts, P = hi + lo (lo = the rounding error of hi, itself
+    // rounded): the products keep ~22 bits of P, so the fp32 accumulation,
+    // not an fp16 rounding of the weights, bounds the error
+    const uint32_t pa0 = pack_half2(pr[0][0], pr[0][1]), pa2 = pack_half2(pr[1][0], pr[1][1]);
+    const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&pa0));
+    const float2 h2 = __half22float2(*reinterpret_cast<const __half2*>(&pa2));
+    const uint32_t pl0 = pack_half2(pr[0][0] - h0.x, pr[0][1] - h0.y);
+    const uint32_t pl2 = pack_half2(pr[1][0] - h2.x, pr[1][1] - h2.y);
+    // ldmatrix.trans: lane l addresses row (l & 7) + 8 ((l >> 3) & 1) of the
+    // slice at feature 8 (l >> 4) of the pair of n tiles
+    const uint32_t vrow = vt + (uint32_t)((lane & 7) + 8 * ((lane >> 3) & 1)) * kRowB + 16 * (lane >> 4);
+#pragma unroll
+    for (int nf = 0; nf < 16; nf += 2) {
+      uint32_t v0, v1, v2, v3;
+      ldsm_x4_trans(vrow + 16 * nf, v0, v1, v2, v3);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        o[nf][e] *= alpha;
+        o[nf + 1][e] *= alpha;
+      }
+      mma_f16(o[nf], pa0, pa2, v0, v1);
+      mma_f16(o[nf], pl0, pl2, v0, v1);
+      mma_f16(o[nf + 1], pa0, pa2, v2, v3);
+      mma_f16(o[nf + 1], pl0, pl2, v2, v3);
     }
     __syncthreads();                                   // the buffer may be refilled
   }
-  if (warp < G) {
-    const size_t slot = ((size_t)m * H + (size_t)kvh * G + warp) * splits + s;
-    *reinterpret_cast<float4*>(part_o + slot * kDh + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-    if (lane == 0) part_ml[slot] = make_float2(mrun, lrun);
+  if (gid < G) {
+    const size_t slot = (((size_t)m * H + (size_t)kvh * G + gid) * splits + s) * kAttnParts + warp;
+    float* dst = part_o + slot * kDh + 2 * tig;
+#pragma unroll
+    for (int nf = 0; nf < 16; ++nf) *reinterpret_cast<float2*>(dst + 8 * nf) = make_float2(o[nf][0], o[nf][1]);
+    if (tig == 0) part_ml[slot] = make_float2(mrun, lrun);
   }
 }
 
@@ -307,7 +373,7 @@ AttnPlan attn_plan(int64_t M, int64_t H, int64_t Hkv, int64_t max_len, int sms) 
   if (sp < 1) sp = 1;
   pl.tiles_per_split = (int)((tiles + sp - 1) / sp);
   pl.splits = (int)((tiles + pl.tiles_per_split - 1) / pl.tiles_per_split);
-  const size_t n = (size_t)M * H * pl.splits;
+  const size_t n = (size_t)M * H * pl.splits * kAttnParts;
   pl.off_ml = (n * kDh * 4 + 255) & ~size_t(255);
   pl.total = pl.off_ml + ((n * 8 + 255) & ~size_t(255));
   return pl;
@@ -355,11 +421,11 @@ cudaError_t launch_attention_decode(const __half* q, const __half* kc, const __h
   }
   float* part_o = static_cast<float*>(ws);
   float2* part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + pl.off_ml);
-  attn_decode_kernel<<<dim3((unsigned)pl.splits, (unsigned)Hkv, (unsigned)M), 256, kAttnSmem, s>>>(
+  attn_decode_kernel<<<dim3((unsigned)pl.splits, (unsigned)Hkv, (unsigned)M), kAttnThreads, kAttnSmem, s>>>(
       q, kc, vc, pos, part_o, part_ml, (int)H, (int)Hkv, (int)Lmax, (int)max_len, pl.tiles_per_split);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<(unsigned)(M * H), kDh, 0, s>>>(part_o, part_ml, out, pl.splits);
+  attn_combine_kernel<<<(unsigned)(M * H), kDh, 0, s>>>(part_o, part_ml, out, pl.splits * kAttnParts);
   return cudaGetLastError();
 }
 
