@@ -104,7 +104,10 @@ __host__ __device__ inline long long cta_of_unit(long long u, long long U, long 
 //    Lanes without a B column read a zero slot.
 template <int M, bool kTQ1> struct Cfg {
   static constexpr int kStages = 4;                       // pairs of weights in flight per warp
-  static constexpr int kWStage = 2048;                    // [block h][row half][32 lanes][16 B]
+  // TQ2: [block h][row half][32 lanes][16 B], then the block scales
+  // [row 0..15][8 B]; TQ1: rows of 112 B, spare words, then the scales
+  static constexpr int kWStage = kTQ1 ? 2048 : 2176;
+  static constexpr int kScaleOff = kTQ1 ? kTq1ScaleOff : 2048;
   static constexpr int kRing = kWarps * kStages * kWStage;
   static constexpr int kLevels = kTQ1 ? 4 : 3;            // activation digit levels per batch row
   static constexpr int kBL = 4 * kLevels * M;             // lanes with a B column (gid < kLevels M)
@@ -241,9 +244,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
   // i = 32 c + lane is chunk i % 7 of row i / 7
   const uint8_t* wrow[4] = {qs, qs, qs, qs};
   uint32_t wsz[4] = {0, 0, 0, 0};
-  const unsigned short* da_p = nullptr;
-  const unsigned short* db_p = nullptr;
-  const unsigned short* ds_p = nullptr;               // TQ1: this lane's scale row, block 2 q_l
+  const unsigned short* ds_p = nullptr;               // this lane's scale row, block 2 q_l
   uint32_t szS = 0;
   const uintptr_t d_end = reinterpret_cast<uintptr_t>(d) + (size_t)p.N * B * 2;
   uint32_t szA = 0, szB = 0;
@@ -265,21 +266,17 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
         wsz[c] = ok ? 16u : 0u;
       }
     }
-    da_p = reinterpret_cast<const unsigned short*>(d) + (size_t)ra * B + 2 * q_l;
-    if constexpr (kTQ1) {
-      // TQ1: lane (gid, tig) copies word tig & 1 of the 8-byte window (from
-      // the 4-byte boundary at or below the pair's two scales) of row
+    {
+      // lane (gid, tig) copies word tig & 1 of the 8-byte window (from the
+      // 4-byte boundary at or below the pair's two scales) of row
       // gid + 8 (tig >> 1)
       const int rowS = rt_l * kRT + warp * 16 + gid + 8 * (tig >> 1);
       szS = rowS < p.N ? 4u : 0u;
       ds_p = reinterpret_cast<const unsigned short*>(d) + (size_t)(szS ? rowS : 0) * B + 2 * q_l;
     }
-    db_p = reinterpret_cast<const unsigned short*>(d) + (size_t)rb * B + 2 * q_l;
   };
   set_rows();
-  // block scales as raw fp16 bits, converted when the stage is consumed (the
-  // loads then have the whole ring depth to land)
-  unsigned short dv[S][2][2];                          // [stage][block h][row half]
+  // weights and block scales of the next unit into ring stage s
   auto issue = [&](int s, bool commit) {
     if (il < n_units) {
       const uint32_t st = ring + s * C::kWStage + lane * 16;
@@ -320,20 +317,12 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
         cp_async_cg16(st + 1024, pa + o1, s1a);
         cp_async_cg16(st + 1536, pb + o1, s1b);
       }
-      if constexpr (kTQ1) {
+      {
         // block scales into the stage's last 128 bytes: [row 0..15][8 bytes]
         const uintptr_t a4 = (reinterpret_cast<uintptr_t>(ds_p) & ~uintptr_t(3)) + 4 * (tig & 1);
         const uint32_t sz = a4 + 4 <= d_end ? szS : (a4 < d_end ? (uint32_t)(d_end - a4) : 0u) * (szS ? 1u : 0u);
-        cp_async_ca4(ring + s * C::kWStage + kTq1ScaleOff + (gid + 8 * (tig >> 1)) * 8 + 4 * (tig & 1),
+        cp_async_ca4(ring + s * C::kWStage + C::kScaleOff + (gid + 8 * (tig >> 1)) * 8 + 4 * (tig & 1),
                      reinterpret_cast<const void*>(a4 < d_end ? a4 : reinterpret_cast<uintptr_t>(d)), sz);
-      } else {
-        // unconditional loads from clamped addresses (a select on the loaded
-        // value would wait for it); rows outside the matrix are never stored
-        // and a missing block has zero weights and zero activation scalars
-        dv[s][0][0] = __ldg(da_p);
-        dv[s][0][1] = __ldg(db_p);
-        dv[s][1][0] = __ldg(da_p + (h1 ? 1 : 0));
-        dv[s][1][1] = __ldg(db_p + (h1 ? 1 : 0));
       }
       ++il;
       if (++q_l == P) {
@@ -343,8 +332,6 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
       } else {
         pa += kPairRow;
         pb += kPairRow;
-        da_p += 2;
-        db_p += 2;
         ds_p += 2;
       }
     }
@@ -548,7 +535,7 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
 #pragma unroll
     for (int m = 0; m < M; ++m) acc[h][m] = 0.f;
   int rt = (int)(u0 / P), q = q0;
-  int seg_q0 = q, j = 0;
+  int j = 0;
   const int r_local = warp * 16 + gid;
   // End of a segment of row tile `tile` that does not cover the whole tile
   // (side 0: it holds the tile's start, i.e. it is this CTA's last segment;
@@ -659,25 +646,28 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
       for (int m = 0; m < M; ++m) acc[h][m] = 0.f;
   };
 
-  if constexpr (kTQ1) {
-    // One unit per iteration with the stage index at run time: the prefix
-    // decode is long, and this keeps one copy of it in the instruction
-    // stream.  The segment ends (row tile ends and the range end) are
-    // handled between the inner loops.
-    // fp16 scale pair of a row from its 8-byte window: the scales start at
-    // byte 2 of it when (row B) is odd
-    const uint32_t dsel = (gid & 1) && (B & 1) ? 0x5432u : 0x3210u;
-    int s = 0;
-    for (int u = 0; u < n_units;) {
-      const int seg_q0 = q, seg_rt = rt;
-      const int seg_len = n_units - u < P - q ? n_units - u : P - q;
+  // One unit per iteration with the stage index at run time, so that the
+  // loop body is emitted once (unrolled over the ring's stages, the body and
+  // the split-tile finish overflowed the instruction cache: ncu counted
+  // 1-2.5 cycles per issued instruction waiting for instructions).  The
+  // segment ends (row tile ends and the range end) are handled between the
+  // inner loops.  fp16 scale pair of a row from its 8-byte window: the
+  // scales start at byte 2 of it when (row B) is odd.
+  const uint32_t dsel = (gid & 1) && (B & 1) ? 0x5432u : 0x3210u;
+  int s = 0;
+  for (int u = 0; u < n_units;) {
+    const int seg_q0 = q, seg_rt = rt;
+    const int seg_len = n_units - u < P - q ? n_units - u : P - q;
 #pragma unroll 1
-      for (int k = 0; k < seg_len; ++k) {
-        cp_async_wait<S - 1>();
-        __syncwarp();                                 // the stage holds other lanes' copies
-        const uint32_t st0 = ring + s * C::kWStage;
+    for (int k = 0; k < seg_len; ++k) {
+      cp_async_wait<S - 1>();
+      __syncwarp();                                   // the scales (and TQ1 rows) are other lanes' copies
+      const uint32_t st0 = ring + s * C::kWStage;
+      // TQ1: words 3 tig .. 3 tig + 2 and 12 of [block h][row gid, gid + 8];
+      // TQ2: this lane's 16 bytes of [block h][row gid, gid + 8]
+      uint32_t tw[2][2][4];
+      if constexpr (kTQ1) {
         const uint32_t r0 = st0 + gid * kTq1RowStride + (kWide ? 8 * (q & 1) : 0);
-        uint32_t tw[2][2][4];                         // [block h][row gid, gid + 8][w0, w1, w2, w12]
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -687,34 +677,49 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
             for (int c3 = 0; c3 < 3; ++c3) tw[h][rr][c3] = ptx::lds32(base + 12 * tig + 4 * c3);
             tw[h][rr][3] = ptx::lds32(base + 48);
           }
-        const uint2 sa = ptx::lds64(st0 + kTq1ScaleOff + gid * 8);
-        const uint2 sb = ptx::lds64(st0 + kTq1ScaleOff + (gid + 8) * 8);
-        __syncwarp();                                 // read: the stage may be refilled
-        issue(s, true);
-        // scales [row half] as (block 0, block 1) fp16 pairs; an odd B's
-        // last pair has one block, whose scale stands in for the missing one
-        // (its weights and activations are zero)
-        const bool h1 = !((B & 1) && q == P - 1);
-        uint32_t dpair[2] = {__byte_perm(sa.x, sa.y, dsel), __byte_perm(sb.x, sb.y, dsel)};
-        if (!h1) {
-          dpair[0] = __byte_perm(dpair[0], 0u, 0x1010);
-          dpair[1] = __byte_perm(dpair[1], 0u, 0x1010);
-        }
-        const uint32_t pj = bfrag + j * C::kPairBytes;
-        const float* sc = reinterpret_cast<const float*>(pair_base + j * C::kPairBytes + 2 * C::kBlkBytes);
+      } else {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint4 bf[4];
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) bf[i] = ptx::lds128(pj + h * C::kBlkBytes + i * C::kBSlots * 16);
-          const uint32_t bw[16] = {bf[0].x, bf[0].y, bf[0].z, bf[0].w, bf[1].x, bf[1].y, bf[1].z, bf[1].w,
-                                   bf[2].x, bf[2].y, bf[2].z, bf[2].w, bf[3].x, bf[3].y, bf[3].z, bf[3].w};
+          for (int rr = 0; rr < 2; ++rr) {
+            const uint4 v = ptx::lds128(st0 + lane * 16 + h * 1024 + rr * 512);
+            tw[h][rr][0] = v.x;
+            tw[h][rr][1] = v.y;
+            tw[h][rr][2] = v.z;
+            tw[h][rr][3] = v.w;
+          }
+      }
+      const uint2 sa = ptx::lds64(st0 + C::kScaleOff + gid * 8);
+      const uint2 sb = ptx::lds64(st0 + C::kScaleOff + (gid + 8) * 8);
+      __syncwarp();                                   // read: the stage may be refilled
+      issue(s, true);
+      // scales [row half] as (block 0, block 1) fp16 pairs; an odd B's last
+      // pair has one block, whose scale stands in for the missing one (its
+      // weights and activations are zero)
+      const bool h1 = !((B & 1) && q == P - 1);
+      uint32_t dpair[2] = {__byte_perm(sa.x, sa.y, dsel), __byte_perm(sb.x, sb.y, dsel)};
+      if (!h1) {
+        dpair[0] = __byte_perm(dpair[0], 0u, 0x1010);
+        dpair[1] = __byte_perm(dpair[1], 0u, 0x1010);
+      }
+      const uint32_t pj = bfrag + j * C::kPairBytes;
+      const float* sc = reinterpret_cast<const float*>(pair_base + j * C::kPairBytes + 2 * C::kBlkBytes);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint4 bf[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bf[i] = ptx::lds128(pj + h * C::kBlkBytes + i * C::kBSlots * 16);
+        const uint32_t bw[16] = {bf[0].x, bf[0].y, bf[0].z, bf[0].w, bf[1].x, bf[1].y, bf[1].z, bf[1].w,
+                                 bf[2].x, bf[2].y, bf[2].z, bf[2].w, bf[3].x, bf[3].y, bf[3].z, bf[3].w};
+        const float da0 = __half2float(__ushort_as_half((unsigned short)(dpair[0] >> (16 * h))));
+        const float da1 = __half2float(__ushort_as_half((unsigned short)(dpair[1] >> (16 * h))));
+        int c[4][4];
+        if constexpr (kTQ1) {
           // prefix registers of rows gid and gid + 8; MMA i takes registers
           // 2i, 2i+1 of each row (chain i % 4)
           uint32_t Aa[16], Ab[16];
           tq1_prefixes(tw[h][0][0], tw[h][0][1], tw[h][0][2], tw[h][0][3], emul, esel, Aa);
           tq1_prefixes(tw[h][1][0], tw[h][1][1], tw[h][1][2], tw[h][1][3], emul, esel, Ab);
-          int c[4][4];
 #pragma unroll
           for (int i = 0; i < 4; ++i)
             mma_u8s8_z(c[i], Aa[2 * i], Ab[2 * i], Aa[2 * i + 1], Ab[2 * i + 1], bw[2 * i], bw[2 * i + 1]);
@@ -734,8 +739,6 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
                     (c[0][2 * r + 1] + c[1][2 * r + 1] + c[2][2 * r + 1] + c[3][2 * r + 1]);
           const int po0 = __shfl_xor_sync(0xFFFFFFFFu, pv[0], 1);
           const int po1 = __shfl_xor_sync(0xFFFFFFFFu, pv[1], 1);
-          const float da0 = __half2float(__ushort_as_half((unsigned short)(dpair[0] >> (16 * h))));
-          const float da1 = __half2float(__ushort_as_half((unsigned short)(dpair[1] >> (16 * h))));
 #pragma unroll
           for (int m = 0; m < M; ++m) {
             const float st = sc[h * 2 * M + m];
@@ -746,87 +749,45 @@ gemv_i8_kernel(const uint8_t* __restrict__ qs, const __half* __restrict__ d, __h
             acc[0][m] = fmaf(own ? (float)s0 : 0.f, st * da0, acc[0][m]);
             acc[1][m] = fmaf(own ? (float)s1 : 0.f, st * da1, acc[1][m]);
           }
-        }
-        s = (s + 1) & (S - 1);
-        if (++j == P) j = 0;                          // slot of pair q: (q - q0) mod P
-        ++q;
-      }
-      u += seg_len;
-      const bool whole = seg_q0 == 0 && q == P;
-      if (q == P) {
-        q = 0;
-        ++rt;
-      }
-      end_segment(seg_rt, whole, seg_q0 == 0 ? 0 : 1);
-    }
-  } else {
-    for (int base = 0; base < n_units; base += S) {
-#pragma unroll
-      for (int s = 0; s < S; ++s) {
-        if (base + s >= n_units) break;
-        cp_async_wait<S - 1>();
-        const uint32_t stg = ring + s * C::kWStage + lane * 16;
-        const uint32_t pj = bfrag + j * C::kPairBytes;
-        const float* sc = reinterpret_cast<const float*>(pair_base + j * C::kPairBytes + 2 * C::kBlkBytes);
-        int c[2][4][4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint4 va = ptx::lds128(stg + h * 1024), vb = ptx::lds128(stg + h * 1024 + 512);
-          uint4 bf[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) bf[i] = ptx::lds128(pj + h * C::kBlkBytes + i * C::kBSlots * 16);
-          const uint32_t bw[16] = {bf[0].x, bf[0].y, bf[0].z, bf[0].w, bf[1].x, bf[1].y, bf[1].z, bf[1].w,
-                                   bf[2].x, bf[2].y, bf[2].z, bf[2].w, bf[3].x, bf[3].y, bf[3].z, bf[3].w};
-          const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
-          const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+        } else {
+          // field g of rows gid (words 0..3 of tw[h][0]) and gid + 8
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const uint32_t mask = 0x03030303u << (2 * g);
-            mma_u8s8_z(c[h][g], wa[0] & mask, wb[0] & mask, wa[1] & mask, wb[1] & mask, bw[g * 2],
-                       bw[g * 2 + 1]);
+            mma_u8s8_z(c[g], tw[h][0][0] & mask, tw[h][1][0] & mask, tw[h][0][1] & mask, tw[h][1][1] & mask,
+                       bw[g * 2], bw[g * 2 + 1]);
           }
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
             const uint32_t mask = 0x03030303u << (2 * g);
-            mma_u8s8(c[h][g], wa[2] & mask, wb[2] & mask, wa[3] & mask, wb[3] & mask, bw[(4 + g) * 2],
-                     bw[(4 + g) * 2 + 1]);
+            mma_u8s8(c[g], tw[h][0][2] & mask, tw[h][1][2] & mask, tw[h][0][3] & mask, tw[h][1][3] & mask,
+                     bw[(4 + g) * 2], bw[(4 + g) * 2 + 1]);
           }
-        }
-        float da[2][2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          da[h][0] = __half2float(__ushort_as_half(dv[s][h][0]));
-          da[h][1] = __half2float(__ushort_as_half(dv[s][h][1]));
-        }
-        // the stage's bytes are in registers (the MMAs consumed them): refill it
-        issue(s, true);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
           float fv[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            fv[e] = (float)(c[h][3][e] + c[h][2][e] * k4 + c[h][1][e] * k16 + c[h][0][e] * k64);
+            fv[e] = (float)(c[3][e] + c[2][e] * k4 + c[1][e] * k16 + c[0][e] * k64);
 #pragma unroll
           for (int m = 0; m < M; ++m) {
             const float st = sc[h * 2 * M + m], nb = wBias[m] * sc[h * 2 * M + M + m];
             const float f0 = fmaf(wA[m], fv[0], fmaf(wB[m], fv[1], nb));
             const float f1 = fmaf(wA[m], fv[2], fmaf(wB[m], fv[3], nb));
-            acc[0][m] = fmaf(f0, st * da[h][0], acc[0][m]);
-            acc[1][m] = fmaf(f1, st * da[h][1], acc[1][m]);
+            acc[0][m] = fmaf(f0, st * da0, acc[0][m]);
+            acc[1][m] = fmaf(f1, st * da1, acc[1][m]);
           }
         }
-
-        const int u = base + s;
-        const int cur_rt = rt, cur_q = q;
-        if (++j == P) j = 0;                            // slot of pair q: (q - q0) mod P
-        if (++q == P) { q = 0; ++rt; }
-        if (cur_q != P - 1 && u != n_units - 1) continue;
-
-        // ------------------------------------------------ end of a row-tile segment
-        end_segment(cur_rt, seg_q0 == 0 && cur_q == P - 1, seg_q0 == 0 ? 0 : 1);
-        seg_q0 = 0;
       }
+      s = (s + 1) & (S - 1);
+      if (++j == P) j = 0;                            // slot of pair q: (q - q0) mod P
+      ++q;
     }
+    u += seg_len;
+    const bool whole = seg_q0 == 0 && q == P;
+    if (q == P) {
+      q = 0;
+      ++rt;
+    }
+    end_segment(seg_rt, whole, seg_q0 == 0 ? 0 : 1);
   }
   cp_async_wait<0>();
   // the last CTA to finish advances the epoch for the next call on this workspace
