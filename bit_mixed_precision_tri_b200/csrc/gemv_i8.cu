@@ -1,6 +1,6 @@
-// Decode-regime ternary GEMV for one or two activation rows (TQ2) on the
-// integer tensor-core path: exact int8 products of the 2-bit weight fields
-// with fixed-point activation digits.
+// Decode-regime ternary GEMV for one or two activation rows on the integer
+// tensor-core path: exact int8 products of the packed weights (TQ2 fields, or
+// TQ1 digit prefixes, see tq1_slot below) with fixed-point activation digits.
 //
 // Y = X (d * W_hat)^T ("Scaling Laws and Efficient Inference for Ternary
 // Language Models", section "The model", step 3).  At M <= 2 the layer is
@@ -31,8 +31,11 @@
 //  * Streaming.  Work = (128-row tile) x (pair of blocks) units split over a
 //    persistent grid as contiguous ranges (stream-K): every CTA streams the
 //    same number of weight bytes.  Each warp owns 16 rows of the tile and
-//    keeps four units of 16-byte cp.async copies in flight, the first four
-//    copied before the wait for the preceding grid.  A row tile split
+//    keeps four units of cp.async copies in flight (weights, and the rows'
+//    block scales in the last 128 bytes of each stage), the first four
+//    copied before the wait for the preceding grid.  The ring is walked with
+//    a run-time stage index, so the loop body exists once in the instruction
+//    stream.  A row tile split
 //    between CTAs is finished by whichever CTA completes its share last:
 //    every contributing warp stores its rows' partial sums, stamped with the
 //    call (one 64-bit store each: no fence), and takes the warp's ticket of
