@@ -342,22 +342,46 @@ attn_decode_kernel(const __half* __restrict__ q, const __half* __restrict__ kc, 
   }
 }
 
-// one CTA of 128 threads per (sequence, query head): sum over the splits
+// One CTA of 128 threads per (sequence, query head) merges the `nparts`
+// partials: the block reduces their maxima, each thread turns a strided share
+// of them into weights exp(max_s - max) in shared memory (dynamic, nparts
+// floats) and sums the weighted row sums; then thread d adds feature d over
+// the partials (coalesced rows of 128 floats).
+__device__ __forceinline__ float block_reduce_128(float v, float* red, bool is_max) {
+  v = is_max ? warp_max(v) : warp_sum(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  const float r = is_max ? fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]))
+                         : (red[0] + red[1]) + (red[2] + red[3]);
+  __syncthreads();                                     // red may be reused
+  return r;
+}
+
 __global__ void __launch_bounds__(128)
 attn_combine_kernel(const float* __restrict__ part_o, const float2* __restrict__ part_ml, __half* __restrict__ out,
-                    int splits) {
+                    int nparts) {
+  extern __shared__ float wsm[];                       // [nparts]
+  __shared__ float red[4];
   const size_t mh = blockIdx.x;
-  const int d = threadIdx.x;
+  const int t = threadIdx.x;
+  const float2* ml = part_ml + mh * nparts;
   float mx = -INFINITY;
-  for (int s = 0; s < splits; ++s) mx = fmaxf(mx, part_ml[mh * splits + s].x);
-  float l = 0.f, acc = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float2 ml = part_ml[mh * splits + s];
-    const float w = ml.y > 0.f ? expf(ml.x - mx) : 0.f;
-    l = fmaf(w, ml.y, l);
-    acc = fmaf(w, part_o[(mh * splits + s) * kDh + d], acc);
+  for (int s = t; s < nparts; s += 128)
+    if (ml[s].y > 0.f) mx = fmaxf(mx, ml[s].x);
+  mx = block_reduce_128(mx, red, true);
+  float l = 0.f;
+  for (int s = t; s < nparts; s += 128) {
+    const float2 v = ml[s];
+    const float w = v.y > 0.f ? expf(v.x - mx) : 0.f;
+    wsm[s] = w;
+    l = fmaf(w, v.y, l);
   }
-  out[mh * kDh + d] = __float2half_rn(acc / l);
+  l = block_reduce_128(l, red, false);                 // its barriers also publish wsm
+  const float* po = part_o + mh * nparts * kDh + t;
+  float acc = 0.f;
+#pragma unroll 4
+  for (int s = 0; s < nparts; ++s) acc = fmaf(wsm[s], po[(size_t)s * kDh], acc);
+  out[mh * kDh + t] = __float2half_rn(acc / l);
 }
 
 struct AttnPlan {
@@ -425,7 +449,8 @@ cudaError_t launch_attention_decode(const __half* q, const __half* kc, const __h
       q, kc, vc, pos, part_o, part_ml, (int)H, (int)Hkv, (int)Lmax, (int)max_len, pl.tiles_per_split);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<(unsigned)(M * H), kDh, 0, s>>>(part_o, part_ml, out, pl.splits * kAttnParts);
+  const int nparts = pl.splits * kAttnParts;           // at most ~2 x SMs x 4: a few KB of weights
+  attn_combine_kernel<<<(unsigned)(M * H), kDh, (size_t)nparts * sizeof(float), s>>>(part_o, part_ml, out, nparts);
   return cudaGetLastError();
 }
 
