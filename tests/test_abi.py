@@ -96,6 +96,39 @@ def test_wait_status_entry_points_reject_bad_arguments(L):
     assert L.tri_selftest_wait_timeout(1, FAKE + 4, None) == 3         # scratch not 8-byte aligned
 
 
+def test_decode_step_entry_points_validate_before_the_device(L):
+    P = FAKE
+    # tri_rmsnorm: nulls, eps, aliasing, shape, alignment
+    assert L.tri_rmsnorm(None, None, P, None, P, 2, 64, 1e-5, None) == 1
+    assert L.tri_rmsnorm(P, P, P, None, P, 2, 64, 1e-5, None) == 1            # residual needs h_out
+    assert L.tri_rmsnorm(P, P + 256, P, P, P, 2, 64, 1e-5, None) == 1         # h_out aliases x
+    assert L.tri_rmsnorm(P, None, P, None, P, 2, 64, -1.0, None) == 1
+    assert L.tri_rmsnorm(P, None, P, None, P, 2, 60, 1e-5, None) == 2          # D % 8
+    assert L.tri_rmsnorm(P, None, P, None, P, 0, 64, 1e-5, None) == 2
+    assert L.tri_rmsnorm(P + 8, None, P, None, P, 2, 64, 1e-5, None) == 3
+    # tri_rope_table
+    assert L.tri_rope_table(None, 16, 128, 5e5, None) == 1
+    assert L.tri_rope_table(P, 16, 128, 1.0, None) == 1                        # theta must exceed 1
+    assert L.tri_rope_table(P, 16, 64, 5e5, None) == 2                         # head dim 128 only
+    assert L.tri_rope_table(P, 0, 128, 5e5, None) == 2
+    assert L.tri_rope_table(P + 4, 16, 128, 5e5, None) == 3
+    # tri_qknorm_rope
+    args = [P, P, P, P, P, P, P, P]
+    assert L.tri_qknorm_rope(*([None] + args[1:]), 1, 8, 2, 16, 1e-5, None) == 1
+    assert L.tri_qknorm_rope(*args, 1, 8, 3, 16, 1e-5, None) == 2             # H % Hkv
+    assert L.tri_qknorm_rope(*args, 1, 8, 2, 0, 1e-5, None) == 2
+    assert L.tri_qknorm_rope(*([P + 8] + args[1:]), 1, 8, 2, 16, 1e-5, None) == 3
+    assert L.tri_qknorm_rope(*(args[:1] + [P + 2] + args[2:]), 1, 8, 2, 16, 1e-5, None) == 3   # pos
+    # tri_attention_decode and its workspace query
+    assert L.tri_attention_decode_workspace_bytes(1, 64, 8, 4096) > 0
+    assert L.tri_attention_decode_workspace_bytes(1, 64, 4, 4096) == 0         # 16 query heads per group
+    assert L.tri_attention_decode_workspace_bytes(1, 64, 8, 0) == 0
+    assert L.tri_attention_decode(None, P, P, P, P, 1, 64, 8, 4096, 4096, P, 1 << 20, None) == 1
+    assert L.tri_attention_decode(P, P, P, P, P, 1, 64, 8, 4096, 4097, P, 1 << 20, None) == 2  # max_len > Lmax
+    assert L.tri_attention_decode(P + 8, P, P, P, P, 1, 64, 8, 4096, 4096, P, 1 << 20, None) == 3   # q
+    assert L.tri_attention_decode(P, P, P, P + 2, P, 1, 64, 8, 4096, 4096, P, 1 << 20, None) == 3   # pos
+
+
 C_PROGRAM = r"""
 #include <stdio.h>
 #include <string.h>
