@@ -18,12 +18,13 @@
 //    features 2l, 2l + 1, 64 + 2l, 65 + 2l: both members of its two pairs.
 //  * attn_decode_kernel: grouped-query attention of each sequence's new
 //    token over its cached positions 0..pos, split over positions.  A CTA
-//    owns (split, key/value head, sequence) and one warp per query head of
-//    the group; 64-position tiles of K and V are double-buffered in shared
-//    memory with cp.async (rows padded to 272 bytes: conflict-free 16-byte
-//    reads), scores and the running softmax are fp32, each lane owns four
-//    output features.  attn_combine_kernel merges the splits' (max, sum,
-//    output) triples.
+//    (4 warps) owns (split, key/value head, sequence); 64-position tiles of
+//    K and V are double-buffered in shared memory with cp.async (rows padded
+//    to 272 bytes: conflict-free fragment reads), and each warp takes 16
+//    positions of every tile: Q K^T and P V on the tensor cores
+//    (mma.sync m16n8k16, fp32 accumulation; the group's query heads are the
+//    A rows), the running softmax in fp32.  attn_combine_kernel merges the
+//    (max, sum, output) triples of every split and warp.
 #include "tri_internal.cuh"
 
 namespace tri {
